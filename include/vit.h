@@ -1,0 +1,169 @@
+/*
+ * vit.h -- C ABI of the B200 (sm_100a) Qwen2-VL native-resolution vision encoder and the
+ * decoder's 3-D M-RoPE position-id builder.
+ *
+ * What the library computes (the passages that define it):
+ *   - "Qwen2-VL" (ZeroModels Keras docs), API, Qwen2VLVisionModel: patch-embed -> rotary blocks
+ *     -> 2x2 merger; Qwen2VLModel table: vision depth 32, width 1280, 16 heads, mlp ratio 4,
+ *     patch 14, spatial merge 2, temporal patch 2, 3 channels, the special token ids and
+ *     mrope_section (16, 24, 24).
+ *   - "Qwen2-VL (Native-Resolution VLM)", Structure table (Patchify 14x14 -> 2D RoPE -> ViT
+ *     blocks -> Patch Merger 2x2) and its exported PatchMerger (LayerNorm, 2x2 group, Linear,
+ *     GELU, Linear).
+ *   - "Qwen2-VL-2B-Instruct -- LiteRT-LM", Conversion notes: packed patches with cu_seqlens,
+ *     per-image full attention, 2-D rope per patch, Conv3d patch embed over 2 frames, the 2x2
+ *     merge of raster patches by strided slices; M-RoPE note (text tokens get 1-D positions).
+ *
+ * Conventions
+ *   - Every tensor argument is caller-owned DEVICE memory unless the comment says "host".
+ *     The library never frees caller memory. bf16 = IEEE bfloat16, row-major, nn.Linear
+ *     weights are [out_features, in_features].
+ *   - Device pointers given to vit_encode / vit_weights_create must be 16-byte aligned
+ *     (the kernels read them with TMA); misaligned pointers return VIT_ERR_ALIGN.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *     default stream) except vit_device_status, which synchronises that stream.
+ *   - Argument errors are returned synchronously, before anything is launched. Errors that
+ *     depend on device data (a malformed M-RoPE prompt, a kernel wait that timed out) are
+ *     written to a device status word and never trap.
+ *   - One handle is used by one stream at a time (its workspace is shared by its calls).
+ */
+#ifndef RESOLUTION_VIT_VISION_B200_VIT_H
+#define RESOLUTION_VIT_VISION_B200_VIT_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------------------------- */
+#define VIT_OK               0
+#define VIT_ERR_ARG          1   /* null pointer, bad size, bad enum value                      */
+#define VIT_ERR_GRID         2   /* grid_thw row with t < 1, or h / w odd or < 2                 */
+#define VIT_ERR_ALIGN        3   /* a device pointer is not 16-byte aligned                      */
+#define VIT_ERR_NOMEM        4   /* workspace allocation failed                                 */
+#define VIT_ERR_CUDA         5   /* a CUDA runtime / driver call failed                         */
+#define VIT_ERR_TOKENS       6   /* (device) M-RoPE prompt malformed: run length != t*h*w/4,
+                                    or a vision run with no grid left                           */
+#define VIT_ERR_TIMEOUT      7   /* (device) a kernel's bounded wait expired; outputs invalid   */
+#define VIT_ERR_UNSUPPORTED  8   /* the current device is not sm_100 (B200 class)               */
+#define VIT_ERR_LIMIT        9   /* a size beyond the library's documented limits               */
+
+/* ---- model constants ("Qwen2-VL", Qwen2VLModel table) -------------------------------------- */
+#define VIT_WIDTH            1280
+#define VIT_HEADS            16
+#define VIT_HEAD_DIM         80
+#define VIT_MLP              5120
+#define VIT_PATCH_DIM        1176   /* 3 channels x 2 frames x 14 x 14, flattened (c, t, ph, pw) */
+#define VIT_MERGE_DIM        5120   /* 2 x 2 x 1280                                               */
+#define VIT_IMAGE_TOKEN_ID        151655
+#define VIT_VIDEO_TOKEN_ID        151656
+#define VIT_VISION_START_TOKEN_ID 151652
+#define VIT_VISION_END_TOKEN_ID   151653
+
+/* ---- limits -------------------------------------------------------------------------------- */
+#define VIT_MAX_IMAGES       512       /* grid_thw rows per vit_encode call                     */
+#define VIT_MAX_SEGMENTS     4096      /* attention segments = sum of t over the images         */
+#define VIT_MAX_PATCHES      (1 << 21) /* patches per vit_encode call                           */
+#define VIT_MAX_SIDE         4096      /* h and w, in patches                                   */
+#define VIT_MAX_MROPE_GRIDS  1024      /* grid_thw rows per mrope_index call                    */
+
+/* ---- weights ------------------------------------------------------------------------------- */
+/* One pre-norm ViT block ("Qwen2-VL (Native-Resolution VLM)", Structure table, ViT Block rows):
+ * all bf16 device pointers. Biases may be NULL (treated as zero); LayerNorm gamma must be given,
+ * beta may be NULL. qkv_w is [3*1280, 1280] with q, k, v stacked in that order, head-major
+ * (head h owns rows h*80 .. h*80+79 of each). */
+typedef struct {
+    const void *ln1_w, *ln1_b;     /* [1280]                 */
+    const void *qkv_w, *qkv_b;     /* [3840, 1280], [3840]   */
+    const void *proj_w, *proj_b;   /* [1280, 1280], [1280]   */
+    const void *ln2_w, *ln2_b;     /* [1280]                 */
+    const void *fc1_w, *fc1_b;     /* [5120, 1280], [5120]   */
+    const void *fc2_w, *fc2_b;     /* [1280, 5120], [1280]   */
+} vit_layer_w;
+
+typedef struct {
+    int depth;                 /* number of ViT blocks, 1..64 (32 for Qwen2-VL)                  */
+    int out_dim;               /* merger output width: a multiple of 16, 16..16384 (1536, 3584)  */
+    float ln_eps;              /* LayerNorm epsilon (1e-6), used by every LayerNorm incl. ln_q   */
+    int patch_order;           /* 0: patches of each frame in 2x2-block order (bh, bw, dh, dw);
+                                  1: raster order (h, w) -- the merge then gathers 2x2 groups    */
+    const void *pe_w;          /* [1280, 1176] patch-embed (Conv3d kernel flattened c,t,ph,pw)   */
+    const void *pe_b;          /* [1280] or NULL                                                */
+    const vit_layer_w *layers; /* HOST array [depth]; copied by vit_weights_create              */
+    const void *lnq_w, *lnq_b; /* merger LayerNorm [1280]                                       */
+    const void *m0_w, *m0_b;   /* merger Linear 1 [5120, 5120], [5120]                          */
+    const void *m2_w, *m2_b;   /* merger Linear 2 [out_dim, 5120], [out_dim]                    */
+} vit_weights_desc;
+
+typedef struct vit_handle vit_handle;  /* validated weight view + workspace + device status word */
+
+/* Validates the descriptor (pointers non-NULL where required, 16-byte aligned, sizes in range),
+ * copies it (not the weight data: the caller keeps the weights alive and unchanged until
+ * vit_weights_destroy) and prepares the tensor maps of the weights on the current device.
+ * Returns VIT_ERR_ARG / VIT_ERR_ALIGN on a bad descriptor (*out untouched), VIT_ERR_CUDA or
+ * VIT_ERR_UNSUPPORTED when no sm_100 device is current. */
+int vit_weights_create(const vit_weights_desc *desc, vit_handle **out);
+
+/* Frees the handle and its workspace. Synchronises the device first. NULL is a no-op. */
+void vit_weights_destroy(vit_handle *h);
+
+/* Host-only: number of patches P = sum t*h*w and merged tokens P/4 for a host grid_thw [n,3].
+ * Validates the grids exactly as vit_encode does. */
+int vit_encode_sizes(const int32_t *grid_thw, int n_images, int64_t *n_patches, int64_t *n_merged);
+
+/* Pre-sizes the handle's workspace for up to max_patches patches (a synchronous allocation).
+ * vit_encode grows the workspace on demand otherwise; call this before capturing vit_encode
+ * into a CUDA graph so that no allocation happens inside the capture. */
+int vit_reserve(vit_handle *h, int64_t max_patches);
+
+/* The encoder forward ("Qwen2-VL", Qwen2VLVisionModel: patch-embed -> rotary blocks -> 2x2
+ * merger). patches: bf16 [P, 1176], the images of grid_thw one after another, each image's
+ * frames in temporal order, each frame's patches in desc.patch_order. grid_thw: HOST int32
+ * [n_images, 3] = (t, h, w) in patch units (h, w even). out: bf16 [P/4, out_dim]; row order =
+ * images in grid_thw order, then t, then the merged (h/2, w/2) grid in raster order.
+ * Attention is full within each (image, frame) segment and never crosses segments.
+ * May allocate (synchronously) if the workspace is too small, see vit_reserve. */
+int vit_encode(const void *patches, const int32_t *grid_thw, int n_images, vit_handle *h,
+               void *out, void *stream);
+
+/* vit_encode with HOST patches and HOST out (pinned memory gives asynchronous copies): copies
+ * the patches into the handle's workspace, encodes, copies the tokens back, all on `stream`.
+ * The host buffers must stay valid until the stream reaches that point. */
+int vit_encode_host(const void *host_patches, const int32_t *grid_thw, int n_images,
+                    vit_handle *h, void *host_out, void *stream);
+
+/* 3-D M-RoPE position ids for the decoder ("Qwen2-VL" intro and Qwen2VLModel table, mrope;
+ * LiteRT-LM card, M-RoPE note). input_ids: int32 [L]. grid_thw: HOST int32 [n_grids, 3], the
+ * grids of the prompt's images and videos in order of appearance (n_grids may be 0; unused
+ * trailing grids are ignored). out: int32 [3, L] (t, h, w axes). delta: int32 [1] or NULL,
+ * receives (largest id + 1) - L. dev_status: int32 [1] or NULL; on a malformed prompt the kernel
+ * writes VIT_ERR_TOKENS there and leaves out/delta untouched (with NULL the error is silent).
+ * The rule: text tokens (incl. vision_start/end) take (c, c, c) from a cursor c that counts up;
+ * a vision run follows a vision_start, is t*(h/2)*(w/2) image or video tokens, its j-th token
+ * takes c + (j / (h'w'), (j / w') % h', j % w'), then c += max(t, h', w').
+ * Host-side returns: VIT_ERR_ARG (NULL pointers, L < 0, n_grids out of range), VIT_ERR_GRID. */
+int mrope_index(const int32_t *input_ids, int64_t L, const int32_t *grid_thw, int n_grids,
+                int32_t *out, int32_t *delta, int32_t *dev_status, void *stream);
+
+/* Synchronises `stream`, reads the handle's device status word into *host_status (VIT_OK or
+ * VIT_ERR_TIMEOUT from a kernel) and clears it. */
+int vit_device_status(vit_handle *h, void *stream, int32_t *host_status);
+
+/* Number of kernels this handle has launched so far (for launch accounting). */
+int64_t vit_launch_count(const vit_handle *h);
+
+/* Per-kernel-class timing with CUDA events recorded on the launch stream around each kernel of
+ * vit_encode. enable != 0 starts recording (clearing earlier totals). vit_profile_read fills
+ * up to n entries of ms_total[] / launches[] in the order of vit_profile_name(i) and returns
+ * the number of classes; it synchronises the stream of the last encode. */
+int vit_profile_enable(vit_handle *h, int enable);
+int vit_profile_read(vit_handle *h, double *ms_total, int64_t *launches, int n);
+const char *vit_profile_name(int i);
+
+const char *vit_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

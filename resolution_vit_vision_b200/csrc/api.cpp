@@ -1,0 +1,567 @@
+// api.cpp -- the C ABI: argument validation, the host-side plan of a packed batch (segments,
+// positions, work lists), the handle's workspace and the launch sequence of vit_encode.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <memory>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "internal.h"
+
+// ============================================================================ device helpers
+namespace vith {
+
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+int g_sms[64] = {};
+}  // namespace
+
+int tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes, uint64_t inner,
+            uint64_t outer, uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+            CUtensorMapSwizzle swizzle) {
+    (void)elem_bytes;
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    if (!g_encode) return VIT_ERR_CUDA;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_pitch_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? VIT_OK : VIT_ERR_CUDA;
+}
+
+int device_sm_count() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && g_sms[dev]) return g_sms[dev];
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+    if (dev < 64) g_sms[dev] = n;
+    return n;
+}
+
+int check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return VIT_ERR_CUDA;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return VIT_ERR_CUDA;
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    return (major == 10 && minor == 0) ? VIT_OK : VIT_ERR_UNSUPPORTED;
+}
+
+}  // namespace vith
+
+// ============================================================================ handle
+namespace {
+
+constexpr int kProfClasses = 10;
+const char *kProfNames[kProfClasses] = {"patch_embed", "layernorm", "qkv_rope", "attention", "out_proj",
+                                        "fc1_gelu",    "fc2",       "merger_fc1", "merger_fc2", "positions"};
+enum ProfClass { P_PE, P_LN, P_QKV, P_ATT, P_PROJ, P_FC1, P_FC2, P_M0, P_M2, P_POS };
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct LayerMaps {
+    CUtensorMap qkv, proj, fc1, fc2;
+};
+
+}  // namespace
+
+struct vit_handle {
+    vit_weights_desc desc{};
+    std::vector<vit_layer_w> layers;
+    std::vector<LayerMaps> maps;
+    CUtensorMap pe_map{}, m0_map{}, m2_map{};
+    int device = 0;
+
+    // workspace
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+    int64_t ws_patches = 0;
+    float *X = nullptr;            // fp32 [P, 1280] residual stream
+    void *H = nullptr;             // bf16 [P, 1280] LayerNorm output / attention output / merger input
+    void *QKV = nullptr;           // bf16 [P, 3840]
+    void *F = nullptr;             // bf16 [P, 5120] fc1 output / merger hidden
+    int32_t *pos = nullptr;        // [P]
+    int32_t *merge_row = nullptr;  // [P]
+    void *patch_stage = nullptr;   // bf16 [P, 1176] (vit_encode_host)
+    void *out_stage = nullptr;     // bf16 [P/4, out_dim] (vit_encode_host)
+    float *rope_cs = nullptr;      // [VIT_MAX_SIDE][20][2]
+    int32_t *status = nullptr;     // device status word
+    bool rope_ready = false;
+
+    // accounting / profiling
+    int64_t launches = 0;
+    bool prof = false;
+    std::vector<cudaEvent_t> ev_pool;
+    std::vector<int> ev_class;     // class of event pair i (events 2i, 2i+1)
+    size_t ev_used = 0;
+    double prof_ms[kProfClasses] = {};
+    int64_t prof_n[kProfClasses] = {};
+    cudaStream_t last_stream = nullptr;
+};
+
+namespace {
+
+int validate_grids(const int32_t *g, int n, int max_n, int64_t *P_out) {
+    if (!g || n < 1 || n > max_n) return VIT_ERR_ARG;
+    int64_t P = 0;
+    for (int i = 0; i < n; ++i) {
+        const int t = g[3 * i], h = g[3 * i + 1], w = g[3 * i + 2];
+        if (t < 1 || h < 2 || w < 2 || (h & 1) || (w & 1)) return VIT_ERR_GRID;
+        if (h > VIT_MAX_SIDE || w > VIT_MAX_SIDE) return VIT_ERR_LIMIT;
+        P += static_cast<int64_t>(t) * h * w;
+        if (P > VIT_MAX_PATCHES) return VIT_ERR_LIMIT;
+    }
+    *P_out = P;
+    return VIT_OK;
+}
+
+// Profiling: an event pair around one launch.
+struct ProfScope {
+    vit_handle *h;
+    cudaStream_t s;
+    int cls;
+    size_t idx = 0;
+    bool on;
+    ProfScope(vit_handle *h_, cudaStream_t s_, int cls_) : h(h_), s(s_), cls(cls_), on(h_ && h_->prof) {
+        if (!on) return;
+        idx = h->ev_used++;
+        while (h->ev_pool.size() < 2 * h->ev_used) {
+            cudaEvent_t e;
+            cudaEventCreate(&e);
+            h->ev_pool.push_back(e);
+        }
+        if (h->ev_class.size() < h->ev_used) h->ev_class.resize(h->ev_used);
+        h->ev_class[idx] = cls;
+        cudaEventRecord(h->ev_pool[2 * idx], s);
+    }
+    ~ProfScope() {
+        if (on) cudaEventRecord(h->ev_pool[2 * idx + 1], s);
+    }
+};
+
+// Fold the recorded event pairs into the per-class totals (synchronises on the last event).
+void prof_collect(vit_handle *h) {
+    if (h->ev_used == 0) return;
+    cudaEventSynchronize(h->ev_pool[2 * (h->ev_used - 1) + 1]);
+    for (size_t i = 0; i < h->ev_used; ++i) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, h->ev_pool[2 * i], h->ev_pool[2 * i + 1]) == cudaSuccess) {
+            h->prof_ms[h->ev_class[i]] += ms;
+            h->prof_n[h->ev_class[i]] += 1;
+        }
+    }
+    h->ev_used = 0;
+}
+
+int ensure_workspace(vit_handle *h, int64_t P) {
+    if (P <= h->ws_patches && h->ws) return VIT_OK;
+    const int64_t Pn = P > 0 ? P : 1;
+    const int out_dim = h->desc.out_dim;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = round_up(off + bytes, 256);
+        return o;
+    };
+    const size_t oX = take(static_cast<size_t>(Pn) * VIT_WIDTH * 4);
+    const size_t oH = take(static_cast<size_t>(Pn) * VIT_WIDTH * 2);
+    const size_t oQKV = take(static_cast<size_t>(Pn) * 3 * VIT_WIDTH * 2);
+    const size_t oF = take(static_cast<size_t>(Pn) * VIT_MLP * 2);
+    const size_t oPos = take(static_cast<size_t>(Pn) * 4);
+    const size_t oMr = take(static_cast<size_t>(Pn) * 4);
+    const size_t oPs = take(static_cast<size_t>(Pn) * VIT_PATCH_DIM * 2);
+    const size_t oOs = take(static_cast<size_t>(Pn / 4 + 1) * out_dim * 2);
+    const size_t oCs = take(static_cast<size_t>(VIT_MAX_SIDE) * 40 * 4);
+    const size_t oSt = take(256);
+    if (h->ws) {
+        cudaDeviceSynchronize();
+        cudaFree(h->ws);
+        h->ws = nullptr;
+    }
+    void *p = nullptr;
+    if (cudaMalloc(&p, off) != cudaSuccess) {
+        cudaGetLastError();
+        h->ws_patches = 0;
+        return VIT_ERR_NOMEM;
+    }
+    uint8_t *b = static_cast<uint8_t *>(p);
+    h->ws = p;
+    h->ws_bytes = off;
+    h->ws_patches = Pn;
+    h->X = reinterpret_cast<float *>(b + oX);
+    h->H = b + oH;
+    h->QKV = b + oQKV;
+    h->F = b + oF;
+    h->pos = reinterpret_cast<int32_t *>(b + oPos);
+    h->merge_row = reinterpret_cast<int32_t *>(b + oMr);
+    h->patch_stage = b + oPs;
+    h->out_stage = b + oOs;
+    h->rope_cs = reinterpret_cast<float *>(b + oCs);
+    h->status = reinterpret_cast<int32_t *>(b + oSt);
+    h->rope_ready = false;
+    if (cudaMemset(h->status, 0, 4) != cudaSuccess) return VIT_ERR_CUDA;
+    return VIT_OK;
+}
+
+#define VIT_TRY(expr)                \
+    do {                             \
+        int _rc = (expr);            \
+        if (_rc != VIT_OK) return _rc; \
+    } while (0)
+
+int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n_images, int64_t P, void *out,
+                  cudaStream_t s) {
+    const vit_weights_desc &d = h->desc;
+    if (h->prof && h->ev_used) prof_collect(h);
+    h->last_stream = s;
+    int64_t &nl = h->launches;
+
+    // host plan: one attention segment per (image, frame)
+    std::vector<int32_t> cu;
+    cu.push_back(0);
+    for (int i = 0; i < n_images; ++i)
+        for (int t = 0; t < grid[3 * i]; ++t) cu.push_back(cu.back() + grid[3 * i + 1] * grid[3 * i + 2]);
+    const int n_seg = static_cast<int>(cu.size()) - 1;
+    if (n_seg > VIT_MAX_SEGMENTS) return VIT_ERR_LIMIT;
+    const int64_t M4 = P / 4;
+
+    if (!h->rope_ready) {
+        ProfScope ps(h, s, P_POS);
+        VIT_TRY(vith::rope_table_launch(h->rope_cs, VIT_MAX_SIDE, s));
+        ++nl;
+        h->rope_ready = true;
+    }
+    {
+        ProfScope ps(h, s, P_POS);
+        VIT_TRY(vith::positions_launch(grid, n_images, P, d.patch_order, h->pos, h->merge_row, s));
+        ++nl;
+    }
+
+    CUtensorMap mPatch, mH, mF, mH4, mF4, mQKV;
+    VIT_TRY(vith::gemm_make_a_map(&mPatch, patches, P, VIT_PATCH_DIM));
+    VIT_TRY(vith::gemm_make_a_map(&mH, h->H, P, VIT_WIDTH));
+    VIT_TRY(vith::gemm_make_a_map(&mF, h->F, P, VIT_MLP));
+    VIT_TRY(vith::gemm_make_a_map(&mH4, h->H, M4, VIT_MERGE_DIM));
+    VIT_TRY(vith::gemm_make_a_map(&mF4, h->F, M4, VIT_MERGE_DIM));
+    VIT_TRY(vith::attn_make_map(&mQKV, h->QKV, P));
+
+    {
+        ProfScope ps(h, s, P_PE);
+        VIT_TRY(vith::gemm_launch(mPatch, h->pe_map, h->X, d.pe_b, P, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32,
+                                  nullptr, nullptr, h->status, s));
+        ++nl;
+    }
+    for (int l = 0; l < d.depth; ++l) {
+        const vit_layer_w &L = h->layers[l];
+        const LayerMaps &lm = h->maps[l];
+        {
+            ProfScope ps(h, s, P_LN);
+            VIT_TRY(vith::layernorm_launch(h->X, L.ln1_w, L.ln1_b, h->H, P, d.ln_eps, nullptr, s));
+            ++nl;
+        }
+        {
+            ProfScope ps(h, s, P_QKV);
+            VIT_TRY(vith::gemm_launch(mH, lm.qkv, h->QKV, L.qkv_b, P, 3 * VIT_WIDTH, VIT_WIDTH, VIT_EPI_QKV_ROPE,
+                                      h->pos, h->rope_cs, h->status, s));
+            ++nl;
+        }
+        {
+            ProfScope ps(h, s, P_ATT);
+            VIT_TRY(vith::attn_launch(mQKV, cu.data(), n_seg, h->H, h->status, s));
+            ++nl;
+        }
+        {
+            ProfScope ps(h, s, P_PROJ);
+            VIT_TRY(vith::gemm_launch(mH, lm.proj, h->X, L.proj_b, P, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32, nullptr,
+                                      nullptr, h->status, s));
+            ++nl;
+        }
+        {
+            ProfScope ps(h, s, P_LN);
+            VIT_TRY(vith::layernorm_launch(h->X, L.ln2_w, L.ln2_b, h->H, P, d.ln_eps, nullptr, s));
+            ++nl;
+        }
+        {
+            ProfScope ps(h, s, P_FC1);
+            VIT_TRY(vith::gemm_launch(mH, lm.fc1, h->F, L.fc1_b, P, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16, nullptr,
+                                      nullptr, h->status, s));
+            ++nl;
+        }
+        {
+            ProfScope ps(h, s, P_FC2);
+            VIT_TRY(vith::gemm_launch(mF, lm.fc2, h->X, L.fc2_b, P, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32, nullptr,
+                                      nullptr, h->status, s));
+            ++nl;
+        }
+    }
+    {
+        ProfScope ps(h, s, P_LN);
+        VIT_TRY(vith::layernorm_launch(h->X, d.lnq_w, d.lnq_b, h->H, P, d.ln_eps,
+                                       d.patch_order == 1 ? h->merge_row : nullptr, s));
+        ++nl;
+    }
+    {
+        ProfScope ps(h, s, P_M0);
+        VIT_TRY(vith::gemm_launch(mH4, h->m0_map, h->F, d.m0_b, M4, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16,
+                                  nullptr, nullptr, h->status, s));
+        ++nl;
+    }
+    {
+        ProfScope ps(h, s, P_M2);
+        VIT_TRY(vith::gemm_launch(mF4, h->m2_map, out, d.m2_b, M4, d.out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16,
+                                  nullptr, nullptr, h->status, s));
+        ++nl;
+    }
+    return VIT_OK;
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+extern "C" {
+
+const char *vit_status_string(int st) {
+    switch (st) {
+        case VIT_OK: return "ok";
+        case VIT_ERR_ARG: return "invalid argument";
+        case VIT_ERR_GRID: return "invalid grid_thw (need t >= 1 and even h, w >= 2)";
+        case VIT_ERR_ALIGN: return "device pointer not 16-byte aligned";
+        case VIT_ERR_NOMEM: return "device allocation failed";
+        case VIT_ERR_CUDA: return "CUDA error";
+        case VIT_ERR_TOKENS: return "malformed M-RoPE prompt (vision run length or grid count)";
+        case VIT_ERR_TIMEOUT: return "a kernel wait timed out";
+        case VIT_ERR_UNSUPPORTED: return "device is not sm_100 (B200 class)";
+        case VIT_ERR_LIMIT: return "size beyond the library limits";
+        default: return "unknown status";
+    }
+}
+
+int vit_encode_sizes(const int32_t *grid_thw, int n_images, int64_t *n_patches, int64_t *n_merged) {
+    if (!n_patches || !n_merged) return VIT_ERR_ARG;
+    int64_t P = 0;
+    const int rc = validate_grids(grid_thw, n_images, VIT_MAX_IMAGES, &P);
+    if (rc != VIT_OK) return rc;
+    *n_patches = P;
+    *n_merged = P / 4;
+    return VIT_OK;
+}
+
+int vit_weights_create(const vit_weights_desc *d, vit_handle **out) {
+    if (!d || !out) return VIT_ERR_ARG;
+    if (d->depth < 1 || d->depth > 64 || d->out_dim < 16 || d->out_dim > 16384 || (d->out_dim % 16) != 0 ||
+        !(d->ln_eps > 0.0f) || (d->patch_order != 0 && d->patch_order != 1) || !d->layers)
+        return VIT_ERR_ARG;
+    const void *req[] = {d->pe_w, d->lnq_w, d->m0_w, d->m2_w};
+    for (const void *p : req)
+        if (!p) return VIT_ERR_ARG;
+    const void *opt[] = {d->pe_w, d->pe_b, d->lnq_w, d->lnq_b, d->m0_w, d->m0_b, d->m2_w, d->m2_b};
+    for (const void *p : opt)
+        if (p && !aligned16(p)) return VIT_ERR_ALIGN;
+    for (int l = 0; l < d->depth; ++l) {
+        const vit_layer_w &L = d->layers[l];
+        const void *lr[] = {L.ln1_w, L.qkv_w, L.proj_w, L.ln2_w, L.fc1_w, L.fc2_w};
+        for (const void *p : lr)
+            if (!p) return VIT_ERR_ARG;
+        const void *la[] = {L.ln1_w, L.ln1_b, L.qkv_w, L.qkv_b, L.proj_w, L.proj_b,
+                            L.ln2_w, L.ln2_b, L.fc1_w, L.fc1_b, L.fc2_w, L.fc2_b};
+        for (const void *p : la)
+            if (p && !aligned16(p)) return VIT_ERR_ALIGN;
+    }
+    int rc = vith::check_device();
+    if (rc != VIT_OK) return rc;
+    std::unique_ptr<vit_handle> h(new (std::nothrow) vit_handle());
+    if (!h) return VIT_ERR_NOMEM;
+    h->desc = *d;
+    h->layers.assign(d->layers, d->layers + d->depth);
+    h->desc.layers = nullptr;
+    cudaGetDevice(&h->device);
+    h->maps.resize(d->depth);
+    rc = vith::gemm_make_b_map(&h->pe_map, d->pe_w, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32);
+    if (rc == VIT_OK) rc = vith::gemm_make_b_map(&h->m0_map, d->m0_w, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16);
+    if (rc == VIT_OK) rc = vith::gemm_make_b_map(&h->m2_map, d->m2_w, d->out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16);
+    for (int l = 0; l < d->depth && rc == VIT_OK; ++l) {
+        const vit_layer_w &L = h->layers[l];
+        LayerMaps &m = h->maps[l];
+        rc = vith::gemm_make_b_map(&m.qkv, L.qkv_w, 3 * VIT_WIDTH, VIT_WIDTH, VIT_EPI_QKV_ROPE);
+        if (rc == VIT_OK) rc = vith::gemm_make_b_map(&m.proj, L.proj_w, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32);
+        if (rc == VIT_OK) rc = vith::gemm_make_b_map(&m.fc1, L.fc1_w, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16);
+        if (rc == VIT_OK) rc = vith::gemm_make_b_map(&m.fc2, L.fc2_w, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32);
+    }
+    if (rc != VIT_OK) return rc;
+    *out = h.release();
+    return VIT_OK;
+}
+
+void vit_weights_destroy(vit_handle *h) {
+    if (!h) return;
+    cudaDeviceSynchronize();
+    for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
+    if (h->ws) cudaFree(h->ws);
+    delete h;
+}
+
+int vit_reserve(vit_handle *h, int64_t max_patches) {
+    if (!h || max_patches < 0) return VIT_ERR_ARG;
+    if (max_patches > VIT_MAX_PATCHES) return VIT_ERR_LIMIT;
+    return ensure_workspace(h, max_patches);
+}
+
+int vit_encode(const void *patches, const int32_t *grid_thw, int n_images, vit_handle *h, void *out, void *stream) {
+    if (!patches || !h || !out) return VIT_ERR_ARG;
+    int64_t P = 0;
+    int rc = validate_grids(grid_thw, n_images, VIT_MAX_IMAGES, &P);
+    if (rc != VIT_OK) return rc;
+    if (!aligned16(patches) || !aligned16(out)) return VIT_ERR_ALIGN;
+    rc = ensure_workspace(h, P);
+    if (rc != VIT_OK) return rc;
+    return encode_device(h, patches, grid_thw, n_images, P, out, static_cast<cudaStream_t>(stream));
+}
+
+int vit_encode_host(const void *host_patches, const int32_t *grid_thw, int n_images, vit_handle *h, void *host_out,
+                    void *stream) {
+    if (!host_patches || !h || !host_out) return VIT_ERR_ARG;
+    int64_t P = 0;
+    int rc = validate_grids(grid_thw, n_images, VIT_MAX_IMAGES, &P);
+    if (rc != VIT_OK) return rc;
+    rc = ensure_workspace(h, P);
+    if (rc != VIT_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t in_bytes = static_cast<size_t>(P) * VIT_PATCH_DIM * 2;
+    const size_t out_bytes = static_cast<size_t>(P / 4) * h->desc.out_dim * 2;
+    if (cudaMemcpyAsync(h->patch_stage, host_patches, in_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return VIT_ERR_CUDA;
+    rc = encode_device(h, h->patch_stage, grid_thw, n_images, P, h->out_stage, s);
+    if (rc != VIT_OK) return rc;
+    if (cudaMemcpyAsync(host_out, h->out_stage, out_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return VIT_ERR_CUDA;
+    return VIT_OK;
+}
+
+int mrope_index(const int32_t *input_ids, int64_t L, const int32_t *grid_thw, int n_grids, int32_t *out,
+                int32_t *delta, int32_t *dev_status, void *stream) {
+    if (L < 0 || n_grids < 0 || n_grids > VIT_MAX_MROPE_GRIDS) return VIT_ERR_ARG;
+    if (L > 0 && (!input_ids || !out)) return VIT_ERR_ARG;
+    if (n_grids > 0 && !grid_thw) return VIT_ERR_ARG;
+    if (L > (int64_t(1) << 30)) return VIT_ERR_LIMIT;
+    for (int i = 0; i < n_grids; ++i) {
+        const int t = grid_thw[3 * i], hh = grid_thw[3 * i + 1], ww = grid_thw[3 * i + 2];
+        if (t < 1 || hh < 2 || ww < 2 || (hh & 1) || (ww & 1)) return VIT_ERR_GRID;
+        if (static_cast<int64_t>(t) * (hh / 2) * (ww / 2) > (int64_t(1) << 30)) return VIT_ERR_LIMIT;
+    }
+    return vith::mrope_launch(input_ids, L, grid_thw, n_grids, out, delta, dev_status,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int vit_device_status(vit_handle *h, void *stream, int32_t *host_status) {
+    if (!h || !host_status) return VIT_ERR_ARG;
+    if (!h->status) {
+        *host_status = VIT_OK;
+        return VIT_OK;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return VIT_ERR_CUDA;
+    int32_t v = 0;
+    if (cudaMemcpy(&v, h->status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return VIT_ERR_CUDA;
+    if (cudaMemset(h->status, 0, 4) != cudaSuccess) return VIT_ERR_CUDA;
+    *host_status = v;
+    return VIT_OK;
+}
+
+int64_t vit_launch_count(const vit_handle *h) { return h ? h->launches : -1; }
+
+int vit_profile_enable(vit_handle *h, int enable) {
+    if (!h) return VIT_ERR_ARG;
+    if (h->ev_used) prof_collect(h);
+    h->prof = enable != 0;
+    for (int i = 0; i < kProfClasses; ++i) {
+        h->prof_ms[i] = 0;
+        h->prof_n[i] = 0;
+    }
+    return VIT_OK;
+}
+
+int vit_profile_read(vit_handle *h, double *ms_total, int64_t *launches, int n) {
+    if (!h) return VIT_ERR_ARG;
+    prof_collect(h);
+    for (int i = 0; i < n && i < kProfClasses; ++i) {
+        if (ms_total) ms_total[i] = h->prof_ms[i];
+        if (launches) launches[i] = h->prof_n[i];
+    }
+    return kProfClasses;
+}
+
+const char *vit_profile_name(int i) { return (i >= 0 && i < kProfClasses) ? kProfNames[i] : nullptr; }
+
+// ---------------------------------------------------------------------------- kernel-level ops
+int vit_op_gemm(const void *A, const void *B, const void *bias, void *C, int64_t M, int N, int K, int epilogue,
+                const int32_t *pos, const float *rope_cs, int32_t *dev_status, void *stream) {
+    if (!A || !B || !C || M < 1 || N < 16 || (N % 16) != 0 || K < 8 || (K % 8) != 0) return VIT_ERR_ARG;
+    if (epilogue < VIT_EPI_STORE_F32 || epilogue > VIT_EPI_QKV_ROPE) return VIT_ERR_ARG;
+    if (epilogue == VIT_EPI_QKV_ROPE && (N != 3 * VIT_WIDTH || !pos || !rope_cs)) return VIT_ERR_ARG;
+    if (M > (int64_t(1) << 30)) return VIT_ERR_LIMIT;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(C) || (bias && !aligned16(bias))) return VIT_ERR_ALIGN;
+    CUtensorMap ta, tb;
+    int rc = vith::gemm_make_a_map(&ta, A, M, K);
+    if (rc == VIT_OK) rc = vith::gemm_make_b_map(&tb, B, N, K, epilogue);
+    if (rc != VIT_OK) return rc;
+    return vith::gemm_launch(ta, tb, C, bias, M, N, K, epilogue, pos, rope_cs, dev_status,
+                             static_cast<cudaStream_t>(stream));
+}
+
+int vit_op_rope_table(float *cs, int n_pos, void *stream) {
+    if (!cs || n_pos < 1 || n_pos > VIT_MAX_SIDE) return VIT_ERR_ARG;
+    return vith::rope_table_launch(cs, n_pos, static_cast<cudaStream_t>(stream));
+}
+
+int vit_op_positions(const int32_t *grid_thw, int n_images, int patch_order, int32_t *pos, int32_t *merge_row,
+                     void *stream) {
+    if (!pos || (patch_order != 0 && patch_order != 1)) return VIT_ERR_ARG;
+    int64_t P = 0;
+    const int rc = validate_grids(grid_thw, n_images, VIT_MAX_IMAGES, &P);
+    if (rc != VIT_OK) return rc;
+    return vith::positions_launch(grid_thw, n_images, P, patch_order, pos, merge_row,
+                                  static_cast<cudaStream_t>(stream));
+}
+
+int vit_op_layernorm(const float *X, const void *gamma, const void *beta, void *Y, int64_t rows, float eps,
+                     const int32_t *out_row, void *stream) {
+    if (!X || !gamma || !Y || rows < 0 || !(eps > 0.0f)) return VIT_ERR_ARG;
+    if (!aligned16(X) || !aligned16(Y) || !aligned16(gamma) || (beta && !aligned16(beta))) return VIT_ERR_ALIGN;
+    return vith::layernorm_launch(X, gamma, beta, Y, rows, eps, out_row, static_cast<cudaStream_t>(stream));
+}
+
+int vit_op_attention(const void *qkv, int64_t P, const int32_t *cu_seqlens, int n_seg, void *out,
+                     int32_t *dev_status, void *stream) {
+    if (!qkv || !out || !cu_seqlens || n_seg < 1 || n_seg > VIT_MAX_SEGMENTS || P < 1) return VIT_ERR_ARG;
+    if (cu_seqlens[0] != 0 || cu_seqlens[n_seg] != P) return VIT_ERR_ARG;
+    for (int i = 0; i < n_seg; ++i)
+        if (cu_seqlens[i + 1] < cu_seqlens[i]) return VIT_ERR_ARG;
+    if (P > VIT_MAX_PATCHES) return VIT_ERR_LIMIT;
+    if (!aligned16(qkv) || !aligned16(out)) return VIT_ERR_ALIGN;
+    CUtensorMap t;
+    const int rc = vith::attn_make_map(&t, qkv, P);
+    if (rc != VIT_OK) return rc;
+    return vith::attn_launch(t, cu_seqlens, n_seg, out, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

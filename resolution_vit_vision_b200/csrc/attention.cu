@@ -1,0 +1,316 @@
+// attention.cu -- varlen, block-diagonal attention on the tcgen05 tensor cores.
+//
+// "Qwen2-VL-2B-Instruct -- LiteRT-LM": the tower uses full attention, one image is one
+// sequence, and the dynamic tower packs all images with cu_seqlens. Here a segment is one
+// (image, frame); every query attends to every key of its own segment and to nothing else:
+// out = softmax(q k^T / sqrt(80)) v per segment and head (16 heads x 80).
+//
+// One CTA = one 128-query tile of one (segment, head). Keys stream through in tiles of 128:
+//   warp 0      TMA producer: Q once, K_j and V_j into a 3-deep ring (32-byte swizzle, the
+//               80-wide head read as five 16-column boxes straight from the [P, 3840] QKV buffer)
+//   warp 1      MMA issuer: S_j = Q K_j^T into one of two TMEM score buffers (M=128, N=128,
+//               K=5x16), then O += P_j V_j (M=128, N=80, K=8x16) into a TMEM output accumulator
+//   warps 2..5  softmax, one query row per thread: scores from TMEM, online max / sum in fp32,
+//               P in bf16 to shared memory (128B-swizzled, K-major), O rescaled in TMEM when the
+//               running max grows, final O / l written as bf16.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <memory>
+#include <vector>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace vitk {
+
+constexpr int kAttnThreads = 192;
+constexpr int kBQ = 128, kBKV = 128, kD = 80;
+constexpr int kKVStages = 3;
+constexpr int kTileBytes = kBQ * kD * 2;          // 20480: 5 boxes of 128 rows x 32 bytes
+constexpr int kBoxBytes = 128 * 32;               // one 16-column box
+constexpr int kPBytes = kBQ * kBKV * 2;           // 32768: two 128B-swizzle atoms of 64 keys
+constexpr int kAttnSmem = 1024 + kTileBytes * (1 + 2 * kKVStages) + kPBytes + 256;
+constexpr int kMaxSegPerLaunch = 512;
+constexpr int kMaxWorkPerLaunch = 4096;
+
+// Work list and segment starts travel as a kernel parameter (no device-side plan buffer).
+struct AttnPlan {
+    int n_work;
+    int n_seg;
+    int start[kMaxSegPerLaunch];      // absolute first row of each segment of this launch
+    int len[kMaxSegPerLaunch];        // its number of rows
+    int work[kMaxWorkPerLaunch];      // (local segment << 16) | q_tile
+};
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ AttnPlan plan,
+                   __nv_bfloat16 *__restrict__ out, int32_t *status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sP = smem;                                   // 32 KB, 1024-aligned (128B swizzle)
+    uint8_t *sQ = sP + kPBytes;
+    uint8_t *sK = sQ + kTileBytes;
+    uint8_t *sV = sK + kKVStages * kTileBytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kKVStages * kTileBytes);
+    uint64_t *q_full = bars;
+    uint64_t *k_full = bars + 1;
+    uint64_t *v_full = k_full + kKVStages;
+    uint64_t *kv_empty = v_full + kKVStages;
+    uint64_t *s_full = kv_empty + kKVStages;     // [2]
+    uint64_t *p_full = s_full + 2;
+    uint64_t *o_done = p_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int item = blockIdx.x / VIT_HEADS, head = blockIdx.x % VIT_HEADS;
+    const int wk = plan.work[item];
+    const int seg = wk >> 16, qt = wk & 0xFFFF;
+    const int seg_start = plan.start[seg], seg_len = plan.len[seg];
+    const int q0 = seg_start + qt * kBQ;
+    const int n_kv = (seg_len + kBKV - 1) / kBKV;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < kKVStages; ++s) {
+            mbar_init(k_full + s, 1);
+            mbar_init(v_full + s, 1);
+            mbar_init(kv_empty + s, 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(s_full + 1, 1);
+        mbar_init(p_full, 128);
+        mbar_init(o_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem;            // two score buffers at columns 0 and 128
+    const uint32_t tO = tmem + 256;      // output accumulator, 80 columns
+    const WaitCtx wc{abort_flag, status};
+
+    if (warp == 0) {
+        if (lane == 0 && seg_len > 0) {
+            tma_prefetch(&tm);
+            mbar_expect_tx(q_full, kTileBytes);
+            for (int c = 0; c < 5; ++c) tma_load_2d(sQ + c * kBoxBytes, &tm, q_full, head * kD + c * 16, q0);
+            for (int j = 0; j < n_kv; ++j) {
+                const int st = j % kKVStages;
+                const uint32_t ph = (j / kKVStages) & 1;
+                if (!mbar_wait(kv_empty + st, ph ^ 1u, wc)) break;
+                const int r0 = seg_start + j * kBKV;
+                mbar_expect_tx(k_full + st, kTileBytes);
+                for (int c = 0; c < 5; ++c)
+                    tma_load_2d(sK + st * kTileBytes + c * kBoxBytes, &tm, k_full + st, VIT_WIDTH + head * kD + c * 16, r0);
+                mbar_expect_tx(v_full + st, kTileBytes);
+                for (int c = 0; c < 5; ++c)
+                    tma_load_2d(sV + st * kTileBytes + c * kBoxBytes, &tm, v_full + st,
+                                2 * VIT_WIDTH + head * kD + c * 16, r0);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && seg_len > 0) {
+            constexpr uint32_t idS = idesc_bf16(kBQ, kBKV, false, false);
+            constexpr uint32_t idO = idesc_bf16(kBQ, kD, false, true);   // V is N(=head dim)-major
+            const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV), pa = smem_u32(sP);
+            bool ok = mbar_wait(q_full, 0, wc);
+            auto issue_s = [&](int j) -> bool {
+                const int st = j % kKVStages;
+                if (!mbar_wait(k_full + st, (j / kKVStages) & 1, wc)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < 5; ++c) {
+                    const uint64_t da = smem_desc(qa + c * kBoxBytes, 16, 256, kSwizzle32B);
+                    const uint64_t db = smem_desc(ka + st * kTileBytes + c * kBoxBytes, 16, 256, kSwizzle32B);
+                    mma_bf16_ss(tS + (j & 1) * 128, da, db, idS, c > 0 ? 1u : 0u);
+                }
+                mma_commit(s_full + (j & 1));
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            if (ok && n_kv > 1) ok = issue_s(1);
+            for (int j = 0; ok && j < n_kv; ++j) {
+                if (!mbar_wait(p_full, j & 1, wc)) break;
+                const int st = j % kKVStages;
+                if (!mbar_wait(v_full + st, (j / kKVStages) & 1, wc)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kBKV / 16; ++kk) {
+                    const uint64_t da = smem_desc(pa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+                    const uint64_t db = smem_desc(va + st * kTileBytes + kk * 512, 4096, 256, kSwizzle32B);
+                    mma_bf16_ss(tO, da, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(kv_empty + st);
+                mma_commit(o_done);
+                if (j + 2 < n_kv) ok = issue_s(j + 2);
+            }
+        }
+    } else if (seg_len > 0) {
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;                          // query row inside the tile
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
+        float m = -INFINITY, l = 0.f;
+        uint8_t *prow = sP + r * 128;
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            if (!mbar_wait(s_full + (j & 1), (j >> 1) & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[128];
+            tmem_ld32(tS + (j & 1) * 128 + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(sr + 0));
+            tmem_ld32(tS + (j & 1) * 128 + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+            tmem_ld32(tS + (j & 1) * 128 + lane_off + 64, *reinterpret_cast<uint32_t(*)[32]>(sr + 64));
+            tmem_ld32(tS + (j & 1) * 128 + lane_off + 96, *reinterpret_cast<uint32_t(*)[32]>(sr + 96));
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) reg_fence32(sr + 32 * c);
+            const int kv_valid = min(kBKV, seg_len - j * kBKV);
+            float x[128];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 128; ++k) {
+                x[k] = (k < kv_valid) ? __uint_as_float(sr[k]) * scale_log2 : -INFINITY;
+                mx = fmaxf(mx, x[k]);
+            }
+            const float m_new = fmaxf(m, mx);
+            const float alpha = ex2(m - m_new);
+            float rs = 0.f;
+#pragma unroll
+            for (int k = 0; k < 128; ++k) {
+                x[k] = ex2(x[k] - m_new);
+                rs += x[k];
+            }
+            l = l * alpha + rs;
+            if (j > 0) {
+                if (!mbar_wait(o_done, (j - 1) & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha < 1.0f)) {
+#pragma unroll
+                    for (int c = 0; c < 5; ++c) {
+                        uint32_t o[16];
+                        tmem_ld16(tO + lane_off + c * 16, o);
+                        tmem_wait_ld();
+                        reg_fence16(o);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st16(tO + lane_off + c * 16, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P row r as bf16 into the 128B-swizzled, K-major tile: 16-byte chunk c of the
+            // 64-key atom goes to chunk c ^ (r % 8)
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const int atom = c >> 3, ch = c & 7;
+                uint4 v = make_uint4(pack_bf16x2(x[8 * c], x[8 * c + 1]), pack_bf16x2(x[8 * c + 2], x[8 * c + 3]),
+                                     pack_bf16x2(x[8 * c + 4], x[8 * c + 5]), pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
+                *reinterpret_cast<uint4 *>(prow + atom * 16384 + ((ch ^ (r & 7)) << 4)) = v;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(p_full);
+            m = m_new;
+        }
+        if (ok && mbar_wait(o_done, (n_kv - 1) & 1, wc)) {
+            tc_fence_after();
+            uint32_t o[80];
+#pragma unroll
+            for (int c = 0; c < 5; ++c) tmem_ld16(tO + lane_off + c * 16, o + c * 16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 5; ++c) reg_fence16(o + c * 16);
+            const int n_q = min(kBQ, seg_len - qt * kBQ);
+            if (r < n_q) {
+                const float inv = 1.0f / l;
+                uint4 *dst = reinterpret_cast<uint4 *>(out + static_cast<int64_t>(q0 + r) * VIT_WIDTH + head * kD);
+#pragma unroll
+                for (int q = 0; q < 10; ++q)
+                    dst[q] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * q]) * inv, __uint_as_float(o[8 * q + 1]) * inv),
+                                        pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv),
+                                        pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv),
+                                        pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) __nanosleep(200000);
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace vitk
+
+namespace vith {
+
+int attn_make_map(CUtensorMap *map, const void *qkv, int64_t P) {
+    return tmap_2d(map, qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * VIT_WIDTH, static_cast<uint64_t>(P),
+                   3 * VIT_WIDTH * 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+// cu_seqlens: HOST [n_seg + 1]. Builds the (segment, q-tile) list, longest segments first,
+// and launches as many kernels as the per-launch limits need.
+int attn_launch(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
+                cudaStream_t s) {
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !configured[dev]) {
+        if (cudaFuncSetAttribute(vitk::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, vitk::kAttnSmem) !=
+            cudaSuccess)
+            return VIT_ERR_CUDA;
+        configured[dev] = true;
+    }
+    // segment order: longest first (longest-processing-time-first over the CTA waves)
+    std::vector<int> order(n_seg);
+    for (int i = 0; i < n_seg; ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+        return (cu_seqlens[a + 1] - cu_seqlens[a]) > (cu_seqlens[b + 1] - cu_seqlens[b]);
+    });
+    auto plan = std::make_unique<vitk::AttnPlan>();
+    size_t pos = 0;
+    while (pos < order.size()) {
+        plan->n_seg = 0;
+        plan->n_work = 0;
+        while (pos < order.size()) {
+            const int sg = order[pos];
+            const int len = cu_seqlens[sg + 1] - cu_seqlens[sg];
+            const int tiles = (len + vitk::kBQ - 1) / vitk::kBQ;
+            if (plan->n_seg == vitk::kMaxSegPerLaunch || plan->n_work + tiles > vitk::kMaxWorkPerLaunch) {
+                if (plan->n_seg == 0) return VIT_ERR_LIMIT;   // one segment alone exceeds a launch
+                break;
+            }
+            const int ls = plan->n_seg++;
+            plan->start[ls] = cu_seqlens[sg];
+            plan->len[ls] = len;
+            for (int t = 0; t < tiles; ++t) plan->work[plan->n_work++] = (ls << 16) | t;
+            ++pos;
+        }
+        if (plan->n_work > 0) {
+            vitk::attn_tc_kernel<<<plan->n_work * VIT_HEADS, vitk::kAttnThreads, vitk::kAttnSmem, s>>>(
+                tqkv, *plan, static_cast<__nv_bfloat16 *>(out), status);
+            if (cudaGetLastError() != cudaSuccess) return VIT_ERR_CUDA;
+        }
+    }
+    return VIT_OK;
+}
+
+}  // namespace vith

@@ -1,0 +1,349 @@
+// gemm.cu -- persistent, warp-specialised tcgen05 GEMM C = A B^T with fused epilogues.
+//
+// Used for every dense contraction of the tower ("Qwen2-VL (Native-Resolution VLM)", Structure
+// table: Patchify 14x14 as a [P,1176]x[1176,1280] product, the ViT blocks' QKV / out-proj /
+// MLP linears, and the Patch Merger's two linears).
+//
+// Per CTA (one per SM, persistent over output tiles of 128 x BN):
+//   warp 0      TMA producer: A and B tiles (128B-swizzled, K-major) into a STAGES-deep ring
+//   warp 1      MMA issuer (one thread): tcgen05.mma 128xBNx16 into a TMEM accumulator;
+//               two accumulators so the epilogue of tile i overlaps the mainloop of tile i+1
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (one row per thread), bias,
+//               GELU / 2-D rope / residual add, stores to global memory
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace vitk {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;           // 64 bf16 = 128 bytes: one 128B swizzle atom per row
+constexpr int kGemmThreads = 192;
+
+template <int BN>
+struct GemmShape {
+    static constexpr int STAGES = 4;
+    static constexpr int A_BYTES = kBM * kBK * 2;
+    static constexpr int B_BYTES = BN * kBK * 2;
+    static constexpr int ACC_STRIDE = 256;    // TMEM columns between the two accumulators
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + 256;
+    static_assert(B_BYTES % 1024 == 0, "B stage must keep 1024-byte alignment");
+};
+
+struct GemmParams {
+    void *C;
+    const __nv_bfloat16 *bias;
+    const int32_t *pos;
+    const float2 *rope_cs;
+    int32_t *status;
+    int M, N, K;
+    int m_tiles, n_tiles, k_blocks;
+};
+
+__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+
+// bias[col0 .. col0+n) -> v (n = 16 or 32; col0 a multiple of 16, bias 16-byte aligned)
+template <int NV>
+__device__ __forceinline__ void add_bias(float *v, const __nv_bfloat16 *bias, int col0) {
+    if (bias == nullptr) return;
+    const uint4 *b4 = reinterpret_cast<const uint4 *>(bias + col0);
+#pragma unroll
+    for (int q = 0; q < NV / 8; ++q) {
+        uint4 u = __ldg(b4 + q);
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[q * 8 + 2 * j] += bf16_lo(w[j]);
+            v[q * 8 + 2 * j + 1] += bf16_hi(w[j]);
+        }
+    }
+}
+
+template <int EPI>
+__device__ __forceinline__ void store_chunk32(const GemmParams &p, int row, int col0, float *v) {
+    if (EPI == VIT_EPI_STORE_F32 || EPI == VIT_EPI_ADD_F32) {
+        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.C) + static_cast<int64_t>(row) * p.N + col0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            float4 o = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            if (EPI == VIT_EPI_ADD_F32) {
+                float4 x = dst[q];
+                o.x += x.x; o.y += x.y; o.z += x.z; o.w += x.w;
+            }
+            dst[q] = o;
+        }
+    } else {
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.C) + static_cast<int64_t>(row) * p.N + col0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float a[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) a[j] = (EPI == VIT_EPI_GELU_BF16) ? gelu_erf(v[8 * q + j]) : v[8 * q + j];
+            dst[q] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                                pack_bf16x2(a[6], a[7]));
+        }
+    }
+}
+
+// columns col0 .. N-1 of a chunk that runs past N (N % 16 == 0, so 16 of the 32 are valid);
+// the loop bound is a compile-time constant so that v stays in registers
+template <int EPI>
+__device__ __forceinline__ void store_partial(const GemmParams &p, int row, int col0, const float *v, int n_valid) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        if (j < n_valid) {
+            float x = v[j];
+            if (p.bias) x += __bfloat162float(p.bias[col0 + j]);
+            const int64_t o = static_cast<int64_t>(row) * p.N + col0 + j;
+            if (EPI == VIT_EPI_STORE_F32) static_cast<float *>(p.C)[o] = x;
+            else if (EPI == VIT_EPI_ADD_F32) static_cast<float *>(p.C)[o] += x;
+            else if (EPI == VIT_EPI_GELU_BF16) static_cast<__nv_bfloat16 *>(p.C)[o] = __float2bfloat16_rn(gelu_erf(x));
+            else static_cast<__nv_bfloat16 *>(p.C)[o] = __float2bfloat16_rn(x);
+        }
+    }
+}
+
+// One 80-wide head of the QKV output: bias, then the 2-D rope on q and k heads (columns < 2560).
+// Pair (d, d+40) turns by the angle of dim d: row position h for d < 20, column w for d >= 20.
+__device__ __forceinline__ void qkv_head(const GemmParams &p, int row, int col0, float *v) {
+    add_bias<80>(v, p.bias, col0);
+    if (col0 < 2 * VIT_WIDTH) {
+        const int hw = p.pos[row];
+        const float2 *ch = p.rope_cs + (hw >> 16) * 20;
+        const float2 *cw = p.rope_cs + (hw & 0xFFFF) * 20;
+#pragma unroll
+        for (int d = 0; d < 40; ++d) {
+            const float2 cs = __ldg(d < 20 ? ch + d : cw + (d - 20));
+            const float x0 = v[d], x1 = v[d + 40];
+            v[d] = x0 * cs.x - x1 * cs.y;
+            v[d + 40] = x1 * cs.x + x0 * cs.y;
+        }
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.C) + static_cast<int64_t>(row) * p.N + col0);
+#pragma unroll
+    for (int q = 0; q < 10; ++q)
+        dst[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                            pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb, GemmParams p) {
+    using S = GemmShape<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + S::STAGES * S::A_BYTES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sB + S::STAGES * S::B_BYTES);
+    uint64_t *empty = full + S::STAGES;
+    uint64_t *tfull = empty + S::STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S::STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull + a, 1);
+            mbar_init(tempty + a, 128);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, S::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const WaitCtx wc{abort_flag, p.status};
+    const int total = p.m_tiles * p.n_tiles;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch(&tma);
+            tma_prefetch(&tmb);
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                const int m0 = (tile / p.n_tiles) * kBM, n0 = (tile % p.n_tiles) * BN;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(empty + stage, phase ^ 1u, wc)) goto producer_done;
+                    mbar_expect_tx(full + stage, S::A_BYTES + S::B_BYTES);
+                    tma_load_2d(sA + stage * S::A_BYTES, &tma, full + stage, kb * kBK, m0);
+                    tma_load_2d(sB + stage * S::B_BYTES, &tmb, full + stage, kb * kBK, n0);
+                    if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+        producer_done:;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(kBM, BN, false, false);
+            int stage = 0;
+            uint32_t phase = 0;
+            int local = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+                const int acc = local & 1;
+                const uint32_t acc_phase = (local >> 1) & 1;
+                if (!mbar_wait(tempty + acc, acc_phase ^ 1u, wc)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * S::ACC_STRIDE;
+                bool ok = true;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(full + stage, phase, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(sA + stage * S::A_BYTES);
+                    const uint32_t b_addr = smem_u32(sB + stage * S::B_BYTES);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        // +32 bytes per 16-element K step inside the 128-byte swizzle atom
+                        const uint64_t da = smem_desc(a_addr + k * 32, 16, 1024, kSwizzle128B);
+                        const uint64_t db = smem_desc(b_addr + k * 32, 16, 1024, kSwizzle128B);
+                        mma_bf16_ss(d_tmem, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(empty + stage);
+                    if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit(tfull + acc);
+            }
+        }
+    } else {
+        const int quarter = warp & 3;   // TMEM lanes [32*quarter, 32*quarter+32) belong to this warp
+        int local = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+            const int acc = local & 1;
+            const uint32_t acc_phase = (local >> 1) & 1;
+            if (!mbar_wait(tfull + acc, acc_phase, wc)) break;
+            tc_fence_after();
+            const int m0 = (tile / p.n_tiles) * kBM, n0 = (tile % p.n_tiles) * BN;
+            const int row = m0 + quarter * 32 + lane;
+            const uint32_t t0 = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * S::ACC_STRIDE;
+            if (EPI == VIT_EPI_QKV_ROPE) {
+#pragma unroll 1
+                for (int hh = 0; hh < BN / 80; ++hh) {
+                    uint32_t r[80];
+#pragma unroll
+                    for (int c = 0; c < 5; ++c) tmem_ld16(t0 + hh * 80 + c * 16, r + c * 16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 5; ++c) reg_fence16(r + c * 16);
+                    float v[80];
+#pragma unroll
+                    for (int j = 0; j < 80; ++j) v[j] = __uint_as_float(r[j]);
+                    if (row < p.M) qkv_head(p, row, n0 + hh * 80, v);
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(t0 + c * 32, r);
+                    tmem_wait_ld();
+                    reg_fence32(r);
+                    const int col0 = n0 + c * 32;
+                    if (row < p.M && col0 < p.N) {
+                        float v[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+                        if (col0 + 32 <= p.N) {
+                            add_bias<32>(v, p.bias, col0);
+                            store_chunk32<EPI>(p, row, col0, v);
+                        } else {
+                            store_partial<EPI>(p, row, col0, v, p.N - col0);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(tempty + acc);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) __nanosleep(200000);   // let copies already in flight land before exit
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, S::TMEM_COLS);
+    }
+}
+
+}  // namespace vitk
+
+namespace vith {
+
+int gemm_make_a_map(CUtensorMap *map, const void *A, int64_t M, int K) {
+    return tmap_2d(map, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, static_cast<uint64_t>(K) * 2, vitk::kBK,
+                   vitk::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue) {
+    const uint32_t bn = (epilogue == VIT_EPI_QKV_ROPE) ? 240 : 256;
+    return tmap_2d(map, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, N, static_cast<uint64_t>(K) * 2, vitk::kBK, bn,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int BN, int EPI>
+static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const vitk::GemmParams &p, cudaStream_t s) {
+    using S = vitk::GemmShape<BN>;
+    static bool configured[64] = {};   // the attribute is set once per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !configured[dev]) {
+        if (cudaFuncSetAttribute(vitk::gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM) !=
+            cudaSuccess)
+            return VIT_ERR_CUDA;
+        if (dev < 64) configured[dev] = true;
+    }
+    const int total = p.m_tiles * p.n_tiles;
+    const int sms = device_sm_count();
+    const int grid = total < sms ? total : sms;
+    vitk::gemm_tc_kernel<BN, EPI><<<grid, vitk::kGemmThreads, S::SMEM, s>>>(ta, tb, p);
+    return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
+}
+
+int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, void *C, const void *bias, int64_t M, int N, int K,
+                int epilogue, const int32_t *pos, const float *rope_cs, int32_t *status, cudaStream_t s) {
+    if (M <= 0) return VIT_OK;
+    vitk::GemmParams p{};
+    p.C = C;
+    p.bias = static_cast<const __nv_bfloat16 *>(bias);
+    p.pos = pos;
+    p.rope_cs = reinterpret_cast<const float2 *>(rope_cs);
+    p.status = status;
+    p.M = static_cast<int>(M);
+    p.N = N;
+    p.K = K;
+    p.m_tiles = static_cast<int>((M + vitk::kBM - 1) / vitk::kBM);
+    p.k_blocks = (K + vitk::kBK - 1) / vitk::kBK;
+    switch (epilogue) {
+        case VIT_EPI_QKV_ROPE:
+            p.n_tiles = N / 240;
+            return launch_one<240, VIT_EPI_QKV_ROPE>(ta, tb, p, s);
+        case VIT_EPI_STORE_F32:
+            p.n_tiles = (N + 255) / 256;
+            return launch_one<256, VIT_EPI_STORE_F32>(ta, tb, p, s);
+        case VIT_EPI_ADD_F32:
+            p.n_tiles = (N + 255) / 256;
+            return launch_one<256, VIT_EPI_ADD_F32>(ta, tb, p, s);
+        case VIT_EPI_STORE_BF16:
+            p.n_tiles = (N + 255) / 256;
+            return launch_one<256, VIT_EPI_STORE_BF16>(ta, tb, p, s);
+        case VIT_EPI_GELU_BF16:
+            p.n_tiles = (N + 255) / 256;
+            return launch_one<256, VIT_EPI_GELU_BF16>(ta, tb, p, s);
+        default:
+            return VIT_ERR_ARG;
+    }
+}
+
+}  // namespace vith

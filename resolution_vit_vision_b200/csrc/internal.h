@@ -1,0 +1,42 @@
+// internal.h -- host-side declarations shared by the C ABI (api.cpp) and the kernel files.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/vit.h"
+#include "../../include/vit_ops.h"
+
+namespace vith {
+
+// ---- tensor maps (driver entry point fetched through the runtime, no -lcuda needed)
+int tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes, uint64_t inner,
+            uint64_t outer, uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+            CUtensorMapSwizzle swizzle);
+
+int device_sm_count();
+int check_device();   // VIT_OK when the current device is sm_100
+
+// ---- GEMM (gemm.cu). A bf16 [M, K], B bf16 [N, K]. The B map may be prebuilt (weights).
+int gemm_make_a_map(CUtensorMap *map, const void *A, int64_t M, int K);
+int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue);
+int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, void *C, const void *bias, int64_t M, int N, int K,
+                int epilogue, const int32_t *pos, const float *rope_cs, int32_t *status, cudaStream_t s);
+
+// ---- attention (attention.cu). qkv bf16 [P, 3840].
+int attn_make_map(CUtensorMap *map, const void *qkv, int64_t P);
+// cu_seqlens: HOST [n_seg + 1]; the (segment, q-tile) work list is built here, longest first
+int attn_launch(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
+                cudaStream_t s);
+
+// ---- small kernels (misc.cu)
+int layernorm_launch(const float *X, const void *gamma, const void *beta, void *Y, int64_t rows, float eps,
+                     const int32_t *out_row, cudaStream_t s);
+int rope_table_launch(float *cs, int n_pos, cudaStream_t s);
+// grid_thw: HOST [n_images, 3] (validated); the table travels as a kernel parameter
+int positions_launch(const int32_t *grid_thw, int n_images, int64_t P, int patch_order, int32_t *pos,
+                     int32_t *merge_row, cudaStream_t s);
+int mrope_launch(const int32_t *ids, int64_t L, const int32_t *grid_thw, int n_grids, int32_t *out, int32_t *delta,
+                 int32_t *status, cudaStream_t s);
+
+}  // namespace vith

@@ -1,0 +1,89 @@
+"""The C-ABI library loads and exports every function include/*.h declares; host-only entry
+points validate their arguments without touching a GPU."""
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from resolution_vit_vision_b200 import build as b
+    if not os.path.exists(b.LIB):
+        b.build()
+    from resolution_vit_vision_b200 import native as nv
+    return nv.lib()
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", src, re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert {"vit_encode", "mrope_index", "vit_weights_create", "vit_op_gemm", "vit_op_attention"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings(lib):
+    from resolution_vit_vision_b200 import native as nv
+    for code in range(10):
+        assert lib.vit_status_string(code)
+    assert b"unknown" in lib.vit_status_string(99)
+
+
+def test_encode_sizes_host_only(lib):
+    from resolution_vit_vision_b200 import native as nv
+    from resolution_vit_vision_b200 import synthetic as syn
+    for wl in syn.WORKLOADS.values():
+        P, M = nv.encode_sizes(wl.grids)
+        assert P == syn.n_patches(wl.grids) and M == P // 4
+    assert nv.encode_sizes([(1, 32, 32)]) == (1024, 256)
+    assert nv.encode_sizes([(1, 48, 48)]) == (2304, 576)
+    for bad, code in [([(1, 7, 8)], nv.VIT_ERR_GRID), ([(0, 8, 8)], nv.VIT_ERR_GRID),
+                      ([(1, 8, 8194)], nv.VIT_ERR_LIMIT)]:
+        with pytest.raises(nv.VitError) as e:
+            nv.encode_sizes(bad)
+        assert e.value.code == code
+
+
+def test_weights_create_rejects_bad_descriptors_before_cuda(lib):
+    from resolution_vit_vision_b200 import native as nv
+    d = nv.VitWeightsDesc()
+    h = ctypes.c_void_p()
+    assert lib.vit_weights_create(None, ctypes.byref(h)) == nv.VIT_ERR_ARG
+    d.depth, d.out_dim, d.ln_eps, d.patch_order = 0, 1536, 1e-6, 0
+    assert lib.vit_weights_create(ctypes.byref(d), ctypes.byref(h)) == nv.VIT_ERR_ARG
+    d.depth, d.out_dim = 1, 1537
+    assert lib.vit_weights_create(ctypes.byref(d), ctypes.byref(h)) == nv.VIT_ERR_ARG
+    layers = (nv.VitLayerW * 1)()
+    d.out_dim, d.layers = 1536, layers
+    assert lib.vit_weights_create(ctypes.byref(d), ctypes.byref(h)) == nv.VIT_ERR_ARG   # null weights
+    fake = 0x10000
+    for k in ("pe_w", "lnq_w", "m0_w", "m2_w"):
+        setattr(d, k, fake)
+    for k in ("ln1_w", "qkv_w", "proj_w", "ln2_w", "fc1_w", "fc2_w"):
+        setattr(layers[0], k, fake)
+    layers[0].qkv_w = fake + 2
+    assert lib.vit_weights_create(ctypes.byref(d), ctypes.byref(h)) == nv.VIT_ERR_ALIGN
+
+
+def test_mrope_rejects_bad_arguments(lib):
+    from resolution_vit_vision_b200 import native as nv
+    g = np.array([[1, 3, 4]], np.int32)
+    assert lib.mrope_index(None, 5, None, 0, None, None, None, None) == nv.VIT_ERR_ARG
+    assert lib.mrope_index(ctypes.c_void_p(16), 5, nv._gp(g), 1, ctypes.c_void_p(16), None, None, None) == nv.VIT_ERR_GRID
+    assert lib.mrope_index(ctypes.c_void_p(16), 5, None, 1, ctypes.c_void_p(16), None, None, None) == nv.VIT_ERR_ARG
+    assert lib.mrope_index(ctypes.c_void_p(16), -1, None, 0, ctypes.c_void_p(16), None, None, None) == nv.VIT_ERR_ARG

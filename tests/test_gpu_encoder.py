@@ -1,0 +1,157 @@
+"""Whole-encoder parity on a B200 through vit_encode (include/vit.h) against the fp64 oracle.
+
+Bar: max|err| <= 3e-2 * max|ref| and per-token cosine >= 0.999 on the bf16 output.
+Full sizes: the 2B-shaped single image at depth 32 is checked whole; the 8-image mixed batch,
+the 1792^2 image and the video batch are checked on outputs the oracle can compute one image at a
+time (block-diagonal attention makes every image independent), in the launch configuration the
+benchmark uses.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import vit_oracle as vo
+from resolution_vit_vision_b200 import native as nv
+from resolution_vit_vision_b200 import synthetic as syn
+from tests.parity import assert_encoder_close, bf16_bits_to_torch, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run(grids, depth, out_dim, seed, order=0, affine=False, patches=None, wts=None):
+    wts = wts if wts is not None else syn.make_weights(depth, out_dim, seed, affine=affine)
+    patches = patches if patches is not None else syn.make_patches(grids, seed)
+    enc = nv.VisionEncoder(nv.weights_to_device(wts), out_dim, 1e-6, order)
+    out = enc.encode(bf16_bits_to_torch(patches), grids)
+    assert enc.device_status() == 0
+    return to_np(out), wts, patches, enc
+
+
+def test_tiny_workload():
+    wl = syn.WORKLOADS["tiny"]
+    got, wts, patches, _ = _run(wl.grids, wl.depth, wl.out_dim, wl.seed)
+    ref = vo.vit_encode(patches, wl.grids, wts)
+    assert got.shape == (16, 1536)
+    assert_encoder_close(got, ref, "tiny")
+
+
+@pytest.mark.parametrize("order", [0, 1])
+def test_ragged_multi_image_affine(order):
+    grids = [(1, 10, 14), (2, 4, 6), (1, 6, 2), (1, 16, 12)]   # 140 + 48 + 12 + 192 = 392 patches
+    got, wts, patches, _ = _run(grids, 2, 1536, 7, order=order, affine=True)
+    ref = vo.vit_encode(patches, grids, wts, patch_order=order)
+    assert_encoder_close(got, ref, f"ragged order {order}")
+
+
+def test_raster_equals_block_order():
+    # T8: the same patches packed raster vs 2x2-block give the same merged tokens
+    grids = [(1, 6, 10), (1, 4, 4)]
+    wts = syn.make_weights(2, 1536, 8)
+    raw = syn.make_patches(grids, 8)              # taken as raster order
+    hp, wp = vo.patch_positions(grids, 0)
+    rows, start = [], 0
+    for t, h, w in grids:
+        fh, fw = vo.frame_positions(h, w, 0)
+        rows.append(start + fh * w + fw)
+        start += h * w
+    block = raw[np.concatenate(rows)]
+    g0, *_ = _run(grids, 2, 1536, 8, order=0, patches=block, wts=wts)
+    g1, *_ = _run(grids, 2, 1536, 8, order=1, patches=raw, wts=wts)
+    assert_encoder_close(g1, g0, "raster vs block")
+
+
+def test_permuting_images_permutes_outputs():
+    # T3 / T4: attention never crosses images, so the order of images only permutes output rows
+    grids = [(1, 8, 8), (1, 4, 12), (1, 10, 6)]
+    wts = syn.make_weights(2, 1536, 9)
+    patches = syn.make_patches(grids, 9)
+    out, *_ = _run(grids, 2, 1536, 9, patches=patches, wts=wts)
+    starts = np.cumsum([0] + [t * h * w for t, h, w in grids])
+    tok = starts // 4
+    perm = [2, 0, 1]
+    p2 = np.concatenate([patches[starts[i]:starts[i + 1]] for i in perm])
+    out2, *_ = _run([grids[i] for i in perm], 2, 1536, 9, patches=p2, wts=wts)
+    ref = np.concatenate([out[tok[i]:tok[i + 1]] for i in perm])
+    np.testing.assert_array_equal(out2, ref)      # same kernels, same per-image work: bit-equal
+    alone, *_ = _run([grids[1]], 2, 1536, 9, patches=patches[starts[1]:starts[2]], wts=wts)
+    np.testing.assert_array_equal(alone, out[tok[1]:tok[2]])
+
+
+def test_encode_host_matches_device():
+    grids = [(1, 8, 12), (1, 6, 6)]
+    got, wts, patches, enc = _run(grids, 2, 1536, 10)
+    hp = torch.from_numpy(patches.copy()).view(torch.bfloat16).pin_memory()
+    ho = torch.empty((got.shape[0], 1536), dtype=torch.bfloat16).pin_memory()
+    enc.encode_host(hp, grids, ho)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(ho.float().numpy(), got)
+
+
+def test_repeat_calls_identical_and_growth():
+    grids = [(1, 8, 8)]
+    wts = syn.make_weights(1, 1536, 11)
+    enc = nv.VisionEncoder(nv.weights_to_device(wts), 1536)
+    p_small = bf16_bits_to_torch(syn.make_patches(grids, 11))
+    a = to_np(enc.encode(p_small, grids))
+    big = [(1, 32, 32), (1, 8, 8)]
+    pb = bf16_bits_to_torch(syn.make_patches(big, 12))
+    enc.encode(pb, big)                            # grows the workspace
+    b = to_np(enc.encode(p_small, grids))
+    np.testing.assert_array_equal(a, b)
+
+
+def test_boundary_errors():
+    wts = syn.make_weights(1, 1536, 13)
+    enc = nv.VisionEncoder(nv.weights_to_device(wts), 1536)
+    p = torch.zeros((64, 1176), dtype=torch.bfloat16, device=DEV)
+    out = torch.zeros((16, 1536), dtype=torch.bfloat16, device=DEV)
+    L = nv.lib()
+    g = np.array([[1, 8, 8]], np.int32)
+    s = torch.cuda.current_stream().cuda_stream
+    assert L.vit_encode(p.data_ptr(), nv._gp(g), 1, enc.handle, None, s) == nv.VIT_ERR_ARG
+    assert L.vit_encode(p.data_ptr(), nv._gp(g), 0, enc.handle, out.data_ptr(), s) == nv.VIT_ERR_ARG
+    for bad in ([1, 7, 8], [0, 8, 8], [1, 8, 0]):
+        gb = np.array([bad], np.int32)
+        assert L.vit_encode(p.data_ptr(), nv._gp(gb), 1, enc.handle, out.data_ptr(), s) == nv.VIT_ERR_GRID
+    assert L.vit_encode(p.data_ptr() + 2, nv._gp(g), 1, enc.handle, out.data_ptr(), s) == nv.VIT_ERR_ALIGN
+    n0 = enc.launch_count()
+    assert L.vit_encode(p.data_ptr(), nv._gp(g), 1, enc.handle, out.data_ptr(), s) == 0
+    assert enc.launch_count() > n0
+
+
+# ------------------------------------------------------------------ full sizes
+@pytest.mark.slow
+def test_2b_448_full_depth():
+    wl = syn.WORKLOADS["2b_448"]
+    got, wts, patches, _ = _run(wl.grids, wl.depth, wl.out_dim, wl.seed)
+    ref = vo.vit_encode(patches, wl.grids, wts)
+    assert got.shape == (256, 1536)
+    assert_encoder_close(got, ref, "2B 448x448 depth 32")
+
+
+@pytest.mark.slow
+def test_mixed8_full_batch_sampled_images():
+    wl = syn.WORKLOADS["mixed8"]
+    got, wts, patches, _ = _run(wl.grids, wl.depth, wl.out_dim, wl.seed)
+    assert got.shape == (4424, 3584)
+    starts = np.cumsum([0] + [t * h * w for t, h, w in wl.grids])
+    for i in (5, 2):      # the 336x336 and the 224x896 images, whole, through the oracle
+        ref = vo.vit_encode(patches[starts[i]:starts[i + 1]], [wl.grids[i]], wts)
+        assert_encoder_close(got[starts[i] // 4:starts[i + 1] // 4], ref, f"mixed8 image {i}")
+    assert np.isfinite(got).all()
+
+
+@pytest.mark.slow
+def test_video_batch_sampled():
+    wl = syn.WORKLOADS["video_2img"]
+    got, wts, patches, _ = _run(wl.grids, wl.depth, wl.out_dim, wl.seed)
+    assert got.shape == (1792, 3584)
+    # the last image, whole
+    s = 4096 + 1536
+    ref = vo.vit_encode(patches[s:], [wl.grids[2]], wts)
+    assert_encoder_close(got[s // 4:], ref, "video batch, image 2")
+    # each frame of the video is its own segment: frame 3 alone equals its rows of the batch
+    one = [(1, 32, 32)]
+    g1, *_ = _run(one, wl.depth, wl.out_dim, wl.seed, patches=patches[3072:4096], wts=wts)
+    np.testing.assert_array_equal(g1, got[768:1024])
