@@ -1,0 +1,362 @@
+"""Benchmark of the B200 Qwen2-VL vision encoder forward (vit_encode) on synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixed8] [--impl reference]
+
+One step = one vit_encode of the whole batch (patch embed, 32 blocks, merger), inputs resident in
+HBM. Default workload: the 8-image mixed-aspect batch (17696 patches, Qwen2-VL-7B-shaped tower,
+out 3584). N > 1 (launched with torch.distributed.run): every rank encodes its own batch (weak
+scaling, no collective on the data path); time = max over ranks of the CUDA-event step time.
+Rank 0 prints one JSON line. ``--impl reference`` times the CPU oracle on a bounded sample of
+the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ViT encode patches/s and merged tokens/s (bf16, 1×B200); % of dense bf16 TC peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mixed8")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--depth", type=int, default=None,
+                    help="override the tower depth (profiling aid: small ncu captures of one layer)")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def ncu_traffic(kernel_class):
+    """DRAM bytes per launch from the committed ncu capture, or None when the kernel's source has
+    changed since the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(p))[kernel_class]
+        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    except (OSError, KeyError, ValueError):
+        return None
+    return rec["bytes_per_launch"] if hashlib.sha1(src).hexdigest() == rec["sha1"] else None
+
+
+# ------------------------------------------------------------------------------ FLOP / byte model
+def segments_of(grids):
+    return [h * w for t, h, w in grids for _ in range(t)]
+
+
+def work_model(grids, depth, out_dim):
+    """Algorithmic FLOPs (2 per multiply-add) and bytes per kernel launch class, per encode."""
+    P = sum(t * h * w for t, h, w in grids)
+    M4 = P // 4
+    s2 = sum(n * n for n in segments_of(grids))
+    per_launch = {
+        "patch_embed": 2.0 * P * 1176 * 1280,
+        "qkv_rope": 2.0 * P * 1280 * 3840,
+        "attention": 4.0 * 1280 * s2,
+        "out_proj": 2.0 * P * 1280 * 1280,
+        "fc1_gelu": 2.0 * P * 1280 * 5120,
+        "fc2": 2.0 * P * 5120 * 1280,
+        "merger_fc1": 2.0 * M4 * 5120 * 5120,
+        "merger_fc2": 2.0 * M4 * 5120 * out_dim,
+    }
+    ln_bytes = P * 1280 * (4 + 2) + 2 * 1280 * 2      # read fp32 row, write bf16 row, gamma/beta
+    total = per_launch["patch_embed"] + per_launch["merger_fc1"] + per_launch["merger_fc2"] + depth * (
+        per_launch["qkv_rope"] + per_launch["attention"] + per_launch["out_proj"] + per_launch["fc1_gelu"] +
+        per_launch["fc2"])
+    return P, M4, per_launch, ln_bytes, total
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join("/tmp", f"vit_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------------------------ CPU baseline (oracle)
+_WCACHE = {}
+
+
+def _oracle_weights(depth, out_dim, seed):
+    from resolution_vit_vision_b200 import synthetic as syn
+    key = (depth, out_dim, seed)
+    if key not in _WCACHE:
+        _WCACHE[key] = syn.make_weights(depth, out_dim, seed)
+    return _WCACHE[key]
+
+
+def cpu_baseline(wl, budget_s=25.0):
+    """The CPU oracle, as it stands, on a bounded sample of the workload: the smallest image of
+    the batch through the full-depth tower (every image is independent, so this is a slice of the
+    same job). Returns patches/s over the sample."""
+    from oracle import vit_oracle as vo
+    from resolution_vit_vision_b200 import synthetic as syn
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        cores = os.cpu_count()
+    i = min(range(len(wl.grids)), key=lambda k: np.prod(wl.grids[k]))
+    g = [wl.grids[i]]
+    P = int(np.prod(g[0]))
+    wts = _oracle_weights(wl.depth, wl.out_dim, wl.seed)
+    patches = syn.make_patches(g, wl.seed)
+    t0 = time.perf_counter()
+    done = 0
+    # a bounded number of passes: at least one, more while under the budget
+    while True:
+        vo.vit_encode(patches, g, wts)
+        done += 1
+        el = time.perf_counter() - t0
+        if el * (done + 1) / done > budget_s:
+            break
+    el = time.perf_counter() - t0
+    return {"value": done * P / el, "unit": "patches/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"image {i} of the batch (grid {tuple(g[0])}, {P} patches) through the full "
+                      f"depth-{wl.depth} fp64 oracle, {done} pass(es), {el:.1f} s"}
+
+
+# ------------------------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from resolution_vit_vision_b200 import synthetic as syn
+    wl = syn.WORKLOADS[args.workload]
+    P, M4, _, _, _ = work_model(wl.grids, wl.depth, wl.out_dim)
+    # each step: one bounded sample (the smallest image of the batch through the full-depth
+    # oracle); the run stops early once about three minutes of CPU time are spent
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(max(1, args.steps)):
+        vals.append(cpu_baseline(wl, budget_s=0.0))
+        if time.perf_counter() - t0 > 180.0:
+            break
+    v = statistics.median(x["value"] for x in vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "patches/s", "n_gpus": args.gpus,
+            "steps": len(vals), "warmup": 0, "ms_per_step": 1000.0 * P / v, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: {wl.description}", "patches": P, "merged": M4,
+                       "depth": wl.depth, "out_dim": wl.out_dim},
+            "merged_tokens_per_s": v / 4,
+            "cpu_baseline": {"value": v, "unit": "patches/s", "cores": vals[0]["cores"], "kind": "oracle",
+                             "sample": vals[0]["sample"]},
+            "e2e": {"value": v, "unit": "patches/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------ native arm
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import torch.distributed as dist
+
+    from resolution_vit_vision_b200 import native as nv
+    from resolution_vit_vision_b200 import synthetic as syn
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    wl = syn.WORKLOADS[args.workload]
+    if args.depth is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, depth=args.depth)
+    P, M4, flops_launch, ln_bytes, flops_total = work_model(wl.grids, wl.depth, wl.out_dim)
+    wts = nv.random_weights_device(wl.depth, wl.out_dim, seed=wl.seed + 17 * rank, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.seed + 1000 + rank)
+    patches = (torch.rand((P, syn.PATCH_K), generator=g, device=dev) * 2 - 1).to(torch.bfloat16)
+    enc = nv.VisionEncoder(wts, wl.out_dim)
+    enc.reserve(P)
+    out = torch.empty((M4, wl.out_dim), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)   # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    clk = None
+    if not args.no_clocks:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        clk = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+        clk.start()
+
+    for _ in range(max(3, args.warmup)):
+        enc.encode(patches, wl.grids, out=out)
+    torch.cuda.synchronize()
+    assert enc.device_status() == 0
+
+    # ---- timed region: K steps, L2 flushed before each, CUDA events per step
+    def timed_steps(profile):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        enc.profile_enable(profile)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        n0 = enc.launch_count()
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            enc.encode(patches, wl.grids, out=out)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        n = enc.launch_count() - n0
+        prof = enc.profile_read() if profile else None
+        enc.profile_enable(False)
+        return float(np.mean([a.elapsed_time(b) for a, b in ev])), n, prof
+
+    ms, launches, _ = timed_steps(False)
+    clocks = clk.stop() if clk else None
+    # the same K steps again with an event pair around every kernel (per-kernel roofline)
+    ms_prof, _, prof = timed_steps(True)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert enc.device_status() == 0
+
+    # ---- e2e: host (pinned) patches in, host tokens out, through vit_encode_host
+    hp = patches.cpu().pin_memory()
+    ho = torch.empty((M4, wl.out_dim), dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        enc.encode_host(hp, wl.grids, ho)
+    torch.cuda.synchronize()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        ev2[i][0].record(stream)
+        enc.encode_host(hp, wl.grids, ho)
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in ev2]))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    pk, pk_kind = peaks()
+    tc_peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    achieved_total = flops_total / (ms * 1e-3) / 1e12
+    kernels = {}
+    for name, rec in prof.items():
+        if rec["launches"] == 0:
+            continue
+        avg = rec["ms"] / rec["launches"]
+        k = {"ms_per_step": rec["ms"] / args.steps, "launches_per_step": rec["launches"] / args.steps,
+             "avg_launch_ms": avg}
+        if name in flops_launch:
+            k["tflops"] = flops_launch[name] / (avg * 1e-3) / 1e12
+            k["frac"] = k["tflops"] / tc_peak
+        elif name == "layernorm":
+            k["gbs"] = ln_bytes / (avg * 1e-3) / 1e9
+            k["frac"] = k["gbs"] / pk["hbm_gbs"]
+        kernels[name] = k
+    top = max((n for n in kernels if n in flops_launch), key=lambda n: kernels[n]["ms_per_step"])
+    roof = {"kernel": top, "bound": "tensor", "achieved": kernels[top]["tflops"], "peak": tc_peak,
+            "unit": "TFLOP/s", "frac": kernels[top]["frac"], "traffic": ncu_traffic(top),
+            "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside the step)"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": world * P / (ms * 1e-3), "unit": "patches/s", "n_gpus": world,
+                "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded random weights N(0,0.02), patches U[-1,1])",
+                "config": {"workload": f"{wl.name}: {wl.description}", "patches": P, "merged": M4,
+                           "depth": wl.depth, "out_dim": wl.out_dim, "l2": "flushed between steps (256 MB write)",
+                           "parallelism": f"dp{world} (images independent; weak scaling)"},
+                "merged_tokens_per_s": world * M4 / (ms * 1e-3),
+                "tc_peak_frac": achieved_total / tc_peak,
+                "tflops": achieved_total,
+                "e2e": {"value": world * P / (e2e_ms * 1e-3), "unit": "patches/s",
+                        "h2d_bytes_per_step": P * syn.PATCH_K * 2, "d2h_bytes_per_step": M4 * wl.out_dim * 2,
+                        "ms_per_step": e2e_ms},
+                "gpu_launches": int(launches),
+                "ms_per_step_profiled": ms_prof,
+                "roofline": roof,
+                "kernels": kernels,
+                "clocks": clocks}
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    enc.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
