@@ -146,6 +146,31 @@ int vit_encode_host(const void *host_patches, const int32_t *grid_thw, int n_ima
 int mrope_index(const int32_t *input_ids, int64_t L, const int32_t *grid_thw, int n_grids,
                 int32_t *out, int32_t *delta, int32_t *dev_status, void *stream);
 
+/* ---- for callers that cannot allocate device memory ----------------------------------------
+ * No counterpart on the pages: this is a deployment variant of vit_encode, not part of the method.
+ * vit_encode keeps its activations in a workspace the handle grows with cudaMalloc. Callers whose
+ * device memory is owned by another allocator, or that forbid device allocation after start-up
+ * (cudaMalloc can synchronise the whole device and can fail at run time), use this instead: it
+ * computes exactly what vit_encode computes, with the activations in a fixed file-scope device
+ * array inside the library, and it calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - Limit: at most VIT_NOALLOC_MAX_PATCHES patches per call (the sum of t*h*w), so the array
+ *     is about 26.3 MB (activations of 1024 patches + the rope table). Every GPU that loads the
+ *     library holds it from load until process exit. Larger batches return VIT_ERR_LIMIT and
+ *     launch nothing.
+ *   - The first call on a device sets the array up on that device (looks up its device address
+ *     and fills its rope table with one kernel on `stream`); make that first call before any
+ *     stream capture.
+ *   - Every call, on every stream, shares the one array and leaves the last call's activations in
+ *     it. Calls whose work overlaps on the GPU race with each other: issue them on one stream or
+ *     order them. Nothing in the array needs clearing between calls: each buffer is fully
+ *     written before it is read.
+ *   - Arguments as for vit_encode; weights from vit_weights_create on the current device.
+ *     dev_status: int32 [1] device or NULL; a kernel wait that timed out writes VIT_ERR_TIMEOUT
+ *     there (it is not cleared by the call). */
+#define VIT_NOALLOC_MAX_PATCHES 1024
+int vit_encode_noalloc(const void *patches, const int32_t *grid_thw, int n_images, vit_handle *weights,
+                       void *out, int32_t *dev_status, void *stream);
+
 /* Synchronises `stream`, reads the handle's device status word into *host_status (VIT_OK or
  * VIT_ERR_TIMEOUT from a kernel) and clears it. */
 int vit_device_status(vit_handle *h, void *stream, int32_t *host_status);

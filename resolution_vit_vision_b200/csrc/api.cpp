@@ -10,6 +10,7 @@
 #include <new>
 #include <vector>
 
+#include "handle.h"
 #include "internal.h"
 
 // ============================================================================ device helpers
@@ -71,53 +72,15 @@ int check_device() {
 // ============================================================================ handle
 namespace {
 
-constexpr int kProfClasses = 10;
-const char *kProfNames[kProfClasses] = {"patch_embed", "layernorm", "qkv_rope", "attention", "out_proj",
+const char *kProfNames[vith::kProfClasses] = {"patch_embed", "layernorm", "qkv_rope", "attention", "out_proj",
                                         "fc1_gelu",    "fc2",       "merger_fc1", "merger_fc2", "positions"};
 enum ProfClass { P_PE, P_LN, P_QKV, P_ATT, P_PROJ, P_FC1, P_FC2, P_M0, P_M2, P_POS };
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-struct LayerMaps {
-    CUtensorMap qkv, proj, fc1, fc2;
-};
-
 }  // namespace
 
-struct vit_handle {
-    vit_weights_desc desc{};
-    std::vector<vit_layer_w> layers;
-    std::vector<LayerMaps> maps;
-    CUtensorMap pe_map{}, m0_map{}, m2_map{};
-    int device = 0;
-
-    // workspace
-    void *ws = nullptr;
-    size_t ws_bytes = 0;
-    int64_t ws_patches = 0;
-    float *X = nullptr;            // fp32 [P, 1280] residual stream
-    void *H = nullptr;             // bf16 [P, 1280] LayerNorm output / attention output / merger input
-    void *QKV = nullptr;           // bf16 [P, 3840]
-    void *F = nullptr;             // bf16 [P, 5120] fc1 output / merger hidden
-    int32_t *pos = nullptr;        // [P]
-    int32_t *merge_row = nullptr;  // [P]
-    void *patch_stage = nullptr;   // bf16 [P, 1176] (vit_encode_host)
-    void *out_stage = nullptr;     // bf16 [P/4, out_dim] (vit_encode_host)
-    float *rope_cs = nullptr;      // [VIT_MAX_SIDE][20][2]
-    int32_t *status = nullptr;     // device status word
-    bool rope_ready = false;
-
-    // accounting / profiling
-    int64_t launches = 0;
-    bool prof = false;
-    std::vector<cudaEvent_t> ev_pool;
-    std::vector<int> ev_class;     // class of event pair i (events 2i, 2i+1)
-    size_t ev_used = 0;
-    double prof_ms[kProfClasses] = {};
-    int64_t prof_n[kProfClasses] = {};
-    cudaStream_t last_stream = nullptr;
-};
 
 namespace {
 
@@ -273,7 +236,7 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
     }
     for (int l = 0; l < d.depth; ++l) {
         const vit_layer_w &L = h->layers[l];
-        const LayerMaps &lm = h->maps[l];
+        const vith::LayerMaps &lm = h->maps[l];
         {
             ProfScope ps(h, s, P_LN);
             VIT_TRY(vith::layernorm_launch(h->X, L.ln1_w, L.ln1_b, h->H, P, d.ln_eps, nullptr, s));
@@ -401,7 +364,7 @@ int vit_weights_create(const vit_weights_desc *d, vit_handle **out) {
     if (rc == VIT_OK) rc = vith::gemm_make_b_map(&h->m2_map, d->m2_w, d->out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16);
     for (int l = 0; l < d->depth && rc == VIT_OK; ++l) {
         const vit_layer_w &L = h->layers[l];
-        LayerMaps &m = h->maps[l];
+        vith::LayerMaps &m = h->maps[l];
         rc = vith::gemm_make_b_map(&m.qkv, L.qkv_w, 3 * VIT_WIDTH, VIT_WIDTH, VIT_EPI_QKV_ROPE);
         if (rc == VIT_OK) rc = vith::gemm_make_b_map(&m.proj, L.proj_w, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32);
         if (rc == VIT_OK) rc = vith::gemm_make_b_map(&m.fc1, L.fc1_w, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16);
@@ -493,7 +456,7 @@ int vit_profile_enable(vit_handle *h, int enable) {
     if (!h) return VIT_ERR_ARG;
     if (h->ev_used) prof_collect(h);
     h->prof = enable != 0;
-    for (int i = 0; i < kProfClasses; ++i) {
+    for (int i = 0; i < vith::kProfClasses; ++i) {
         h->prof_ms[i] = 0;
         h->prof_n[i] = 0;
     }
@@ -503,14 +466,14 @@ int vit_profile_enable(vit_handle *h, int enable) {
 int vit_profile_read(vit_handle *h, double *ms_total, int64_t *launches, int n) {
     if (!h) return VIT_ERR_ARG;
     prof_collect(h);
-    for (int i = 0; i < n && i < kProfClasses; ++i) {
+    for (int i = 0; i < n && i < vith::kProfClasses; ++i) {
         if (ms_total) ms_total[i] = h->prof_ms[i];
         if (launches) launches[i] = h->prof_n[i];
     }
-    return kProfClasses;
+    return vith::kProfClasses;
 }
 
-const char *vit_profile_name(int i) { return (i >= 0 && i < kProfClasses) ? kProfNames[i] : nullptr; }
+const char *vit_profile_name(int i) { return (i >= 0 && i < vith::kProfClasses) ? kProfNames[i] : nullptr; }
 
 // ---------------------------------------------------------------------------- kernel-level ops
 int vit_op_gemm(const void *A, const void *B, const void *bias, void *C, int64_t M, int N, int K, int epilogue,

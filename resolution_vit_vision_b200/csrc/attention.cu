@@ -313,4 +313,52 @@ int attn_launch(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, v
     return VIT_OK;
 }
 
+// attn_launch with the schedule kept on the host stack and an in-place sort (ties broken by
+// segment index, the order attn_launch's stable sort gives), for callers that must not allocate.
+int attn_launch_stack(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
+                      cudaStream_t s) {
+    if (n_seg < 0 || n_seg > VIT_MAX_SEGMENTS) return VIT_ERR_LIMIT;
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !configured[dev]) {
+        if (cudaFuncSetAttribute(vitk::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, vitk::kAttnSmem) !=
+            cudaSuccess)
+            return VIT_ERR_CUDA;
+        if (dev < 64) configured[dev] = true;
+    }
+    int order[VIT_MAX_SEGMENTS];
+    for (int i = 0; i < n_seg; ++i) order[i] = i;
+    std::sort(order, order + n_seg, [&](int a, int b) {
+        const int la = cu_seqlens[a + 1] - cu_seqlens[a], lb = cu_seqlens[b + 1] - cu_seqlens[b];
+        return la != lb ? la > lb : a < b;
+    });
+    vitk::AttnPlan plan;
+    int pos = 0;
+    while (pos < n_seg) {
+        plan.n_seg = 0;
+        plan.n_work = 0;
+        while (pos < n_seg) {
+            const int sg = order[pos];
+            const int len = cu_seqlens[sg + 1] - cu_seqlens[sg];
+            const int tiles = (len + vitk::kBQ - 1) / vitk::kBQ;
+            if (plan.n_seg == vitk::kMaxSegPerLaunch || plan.n_work + tiles > vitk::kMaxWorkPerLaunch) {
+                if (plan.n_seg == 0) return VIT_ERR_LIMIT;
+                break;
+            }
+            const int ls = plan.n_seg++;
+            plan.start[ls] = cu_seqlens[sg];
+            plan.len[ls] = len;
+            for (int t = 0; t < tiles; ++t) plan.work[plan.n_work++] = (ls << 16) | t;
+            ++pos;
+        }
+        if (plan.n_work > 0) {
+            vitk::attn_tc_kernel<<<plan.n_work * VIT_HEADS, vitk::kAttnThreads, vitk::kAttnSmem, s>>>(
+                tqkv, plan, static_cast<__nv_bfloat16 *>(out), status);
+            if (cudaGetLastError() != cudaSuccess) return VIT_ERR_CUDA;
+        }
+    }
+    return VIT_OK;
+}
+
 }  // namespace vith

@@ -1,0 +1,51 @@
+// handle.h -- the vit_handle behind the C ABI: the validated weight view (descriptor copy and
+// the weights' TMA descriptors), the lazily grown workspace and the profiling state.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "../../include/vit.h"
+
+namespace vith {
+struct LayerMaps {
+    CUtensorMap qkv, proj, fc1, fc2;
+};
+constexpr int kProfClasses = 10;
+}  // namespace vith
+
+struct vit_handle {
+    vit_weights_desc desc{};
+    std::vector<vit_layer_w> layers;
+    std::vector<vith::LayerMaps> maps;
+    CUtensorMap pe_map{}, m0_map{}, m2_map{};
+    int device = 0;
+
+    // workspace
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+    int64_t ws_patches = 0;
+    float *X = nullptr;            // fp32 [P, 1280] residual stream
+    void *H = nullptr;             // bf16 [P, 1280] LayerNorm output / attention output / merger input
+    void *QKV = nullptr;           // bf16 [P, 3840]
+    void *F = nullptr;             // bf16 [P, 5120] fc1 output / merger hidden
+    int32_t *pos = nullptr;        // [P]
+    int32_t *merge_row = nullptr;  // [P]
+    void *patch_stage = nullptr;   // bf16 [P, 1176] (vit_encode_host)
+    void *out_stage = nullptr;     // bf16 [P/4, out_dim] (vit_encode_host)
+    float *rope_cs = nullptr;      // [VIT_MAX_SIDE][20][2]
+    int32_t *status = nullptr;     // device status word
+    bool rope_ready = false;
+
+    // accounting / profiling
+    int64_t launches = 0;
+    bool prof = false;
+    std::vector<cudaEvent_t> ev_pool;
+    std::vector<int> ev_class;     // class of event pair i (events 2i, 2i+1)
+    size_t ev_used = 0;
+    double prof_ms[vith::kProfClasses] = {};
+    int64_t prof_n[vith::kProfClasses] = {};
+    cudaStream_t last_stream = nullptr;
+};

@@ -36,6 +36,11 @@ int rope_table_launch(float *cs, int n_pos, cudaStream_t s);
 // grid_thw: HOST [n_images, 3] (validated); the table travels as a kernel parameter
 int positions_launch(const int32_t *grid_thw, int n_images, int64_t P, int patch_order, int32_t *pos,
                      int32_t *merge_row, cudaStream_t s);
+// the same launches with their host-side tables on the stack (no heap use)
+int attn_launch_stack(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
+                      cudaStream_t s);
+int positions_launch_stack(const int32_t *grid_thw, int n_images, int64_t P, int patch_order, int32_t *pos,
+                           int32_t *merge_row, cudaStream_t s);
 int mrope_launch(const int32_t *ids, int64_t L, const int32_t *grid_thw, int n_grids, int32_t *out, int32_t *delta,
                  int32_t *status, cudaStream_t s);
 

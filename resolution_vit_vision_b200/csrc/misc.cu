@@ -284,6 +284,26 @@ int positions_launch(const int32_t *grid_thw, int n_images, int64_t P, int patch
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 
+// positions_launch with the image table on the host stack, for callers that must not allocate.
+int positions_launch_stack(const int32_t *grid_thw, int n_images, int64_t P, int patch_order, int32_t *pos,
+                           int32_t *merge_row, cudaStream_t s) {
+    if (n_images < 0 || n_images > VIT_MAX_IMAGES) return VIT_ERR_LIMIT;
+    vitk::ImageTable tab;
+    tab.n = n_images;
+    int64_t row = 0;
+    for (int i = 0; i < n_images; ++i) {
+        tab.row_start[i] = static_cast<int>(row);
+        tab.t[i] = grid_thw[3 * i];
+        tab.h[i] = grid_thw[3 * i + 1];
+        tab.w[i] = grid_thw[3 * i + 2];
+        row += static_cast<int64_t>(tab.t[i]) * tab.h[i] * tab.w[i];
+    }
+    if (P <= 0) return VIT_OK;
+    vitk::positions_kernel<<<static_cast<unsigned>((P + 255) / 256), 256, 0, s>>>(tab, P, patch_order, pos,
+                                                                                 merge_row);
+    return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
+}
+
 int mrope_launch(const int32_t *ids, int64_t L, const int32_t *grid_thw, int n_grids, int32_t *out, int32_t *delta,
                  int32_t *status, cudaStream_t s) {
     auto g = std::make_unique<vitk::MropeGrids>();

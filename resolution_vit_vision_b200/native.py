@@ -45,6 +45,7 @@ _SIGS = {
     "vit_reserve": (c_int, [c_void_p, c_int64]),
     "vit_encode": (c_int, [c_void_p, c_i32p, c_int, c_void_p, c_void_p, c_void_p]),
     "vit_encode_host": (c_int, [c_void_p, c_i32p, c_int, c_void_p, c_void_p, c_void_p]),
+    "vit_encode_noalloc": (c_int, [c_void_p, c_i32p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "mrope_index": (c_int, [c_void_p, c_int64, c_i32p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "vit_device_status": (c_int, [c_void_p, c_void_p, c_i32p]),
     "vit_launch_count": (c_int64, [c_void_p]),
