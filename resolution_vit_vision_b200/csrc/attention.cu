@@ -24,15 +24,18 @@
 
 namespace vitk {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;                 // 10 warps
 constexpr int kBQ = 128, kBKV = 128, kD = 80;
+constexpr int kQTilesPerCta = 2;                  // query tiles A and B share every K/V tile
 constexpr int kKVStages = 3;
 constexpr int kTileBytes = kBQ * kD * 2;          // 20480: 5 boxes of 128 rows x 32 bytes
 constexpr int kBoxBytes = 128 * 32;               // one 16-column box
-constexpr int kPBytes = kBQ * kBKV * 2;           // 32768: two 128B-swizzle atoms of 64 keys
-constexpr int kAttnSmem = 1024 + kTileBytes * (1 + 2 * kKVStages) + kPBytes + 256;
+constexpr int kAttnSmem = 1024 + kTileBytes * (kQTilesPerCta + 2 * kKVStages) + 256;
 constexpr int kMaxSegPerLaunch = 512;
 constexpr int kMaxWorkPerLaunch = 4096;
+// Lazy rescaling: the exponent offset of a row only moves when its running max grows by more
+// than this (log2 units), so P stays below 2^8 and O is rarely rescaled.
+constexpr float kRescaleThreshold = 8.0f;
 
 // Work list and segment starts travel as a kernel parameter (no device-side plan buffer).
 struct AttnPlan {
@@ -40,7 +43,7 @@ struct AttnPlan {
     int n_seg;
     int start[kMaxSegPerLaunch];      // absolute first row of each segment of this launch
     int len[kMaxSegPerLaunch];        // its number of rows
-    int work[kMaxWorkPerLaunch];      // (local segment << 16) | q_tile
+    int work[kMaxWorkPerLaunch];      // (local segment << 16) | pair of query tiles
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -49,32 +52,35 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// TMEM columns: S_A / P_A at 0, S_B / P_B at 128 (P, bf16 pairs, overwrites the first 64 columns
+// of its S once the scores are in registers), O_A at 256, O_B at 384 (80 columns each).
+// 10 warps put 3 warps on two of the SM's four sub-partitions (16K registers each), which caps
+// a thread at 168 registers.
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ AttnPlan plan,
                    __nv_bfloat16 *__restrict__ out, int32_t *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sP = smem;                                   // 32 KB, 1024-aligned (128B swizzle)
-    uint8_t *sQ = sP + kPBytes;
-    uint8_t *sK = sQ + kTileBytes;
+    uint8_t *sQ = smem;                                   // [2][5 boxes]
+    uint8_t *sK = sQ + kQTilesPerCta * kTileBytes;
     uint8_t *sV = sK + kKVStages * kTileBytes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kKVStages * kTileBytes);
     uint64_t *q_full = bars;
     uint64_t *k_full = bars + 1;
     uint64_t *v_full = k_full + kKVStages;
     uint64_t *kv_empty = v_full + kKVStages;
-    uint64_t *s_full = kv_empty + kKVStages;     // [2]
-    uint64_t *p_full = s_full + 2;
-    uint64_t *o_done = p_full + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 1);
+    uint64_t *s_full = kv_empty + kKVStages;     // [2] per query tile
+    uint64_t *p_full = s_full + 2;               // [2]
+    uint64_t *o_done = p_full + 2;               // [2]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int item = blockIdx.x / VIT_HEADS, head = blockIdx.x % VIT_HEADS;
     const int wk = plan.work[item];
-    const int seg = wk >> 16, qt = wk & 0xFFFF;
+    const int seg = wk >> 16, pair = wk & 0xFFFF;
     const int seg_start = plan.start[seg], seg_len = plan.len[seg];
-    const int q0 = seg_start + qt * kBQ;
+    const int q0 = seg_start + pair * kQTilesPerCta * kBQ;
     const int n_kv = (seg_len + kBKV - 1) / kBKV;
 
     if (threadIdx.x == 0) {
@@ -84,10 +90,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(v_full + s, 1);
             mbar_init(kv_empty + s, 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(s_full + 1, 1);
-        mbar_init(p_full, 128);
-        mbar_init(o_done, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(s_full + x, 1);
+            mbar_init(p_full + x, 128);
+            mbar_init(o_done + x, 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -99,15 +106,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem;            // two score buffers at columns 0 and 128
-    const uint32_t tO = tmem + 256;      // output accumulator, 80 columns
     const WaitCtx wc{abort_flag, status};
 
     if (warp == 0) {
         if (lane == 0 && seg_len > 0) {
             tma_prefetch(&tm);
-            mbar_expect_tx(q_full, kTileBytes);
-            for (int c = 0; c < 5; ++c) tma_load_2d(sQ + c * kBoxBytes, &tm, q_full, head * kD + c * 16, q0);
+            mbar_expect_tx(q_full, kQTilesPerCta * kTileBytes);
+            for (int x = 0; x < kQTilesPerCta; ++x)
+                for (int c = 0; c < 5; ++c)
+                    tma_load_2d(sQ + x * kTileBytes + c * kBoxBytes, &tm, q_full, head * kD + c * 16, q0 + x * kBQ);
             for (int j = 0; j < n_kv; ++j) {
                 const int st = j % kKVStages;
                 const uint32_t ph = (j / kKVStages) & 1;
@@ -126,118 +133,142 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0 && seg_len > 0) {
             constexpr uint32_t idS = idesc_bf16(kBQ, kBKV, false, false);
             constexpr uint32_t idO = idesc_bf16(kBQ, kD, false, true);   // V is N(=head dim)-major
-            const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV), pa = smem_u32(sP);
-            bool ok = mbar_wait(q_full, 0, wc);
-            auto issue_s = [&](int j) -> bool {
+            const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
+            // S_x(j) = Q_x K_j^T into TMEM columns 128 x
+            auto issue_s = [&](int x, int j) {
                 const int st = j % kKVStages;
-                if (!mbar_wait(k_full + st, (j / kKVStages) & 1, wc)) return false;
-                tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < 5; ++c) {
-                    const uint64_t da = smem_desc(qa + c * kBoxBytes, 16, 256, kSwizzle32B);
+                    const uint64_t da = smem_desc(qa + x * kTileBytes + c * kBoxBytes, 16, 256, kSwizzle32B);
                     const uint64_t db = smem_desc(ka + st * kTileBytes + c * kBoxBytes, 16, 256, kSwizzle32B);
-                    mma_bf16_ss(tS + (j & 1) * 128, da, db, idS, c > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + x * 128, da, db, idS, c > 0 ? 1u : 0u);
                 }
-                mma_commit(s_full + (j & 1));
-                return true;
+                mma_commit(s_full + x);
             };
-            if (ok) ok = issue_s(0);
-            if (ok && n_kv > 1) ok = issue_s(1);
-            for (int j = 0; ok && j < n_kv; ++j) {
-                if (!mbar_wait(p_full, j & 1, wc)) break;
+            // O_x += P_x(j) V_j, P_x read from TMEM (8 columns per 16 keys)
+            auto issue_pv = [&](int x, int j) {
                 const int st = j % kKVStages;
-                if (!mbar_wait(v_full + st, (j / kKVStages) & 1, wc)) break;
-                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kBKV / 16; ++kk) {
-                    const uint64_t da = smem_desc(pa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128B);
                     const uint64_t db = smem_desc(va + st * kTileBytes + kk * 512, 4096, 256, kSwizzle32B);
-                    mma_bf16_ss(tO, da, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
                 }
+                mma_commit(o_done + x);
+            };
+            bool ok = mbar_wait(q_full, 0, wc) && mbar_wait(k_full, 0, wc);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                issue_s(1, 0);
+            }
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int st = j % kKVStages;
+                const uint32_t ph = j & 1;
+                const bool more = j + 1 < n_kv;
+                const int st1 = (j + 1) % kKVStages;
+                if (!mbar_wait(p_full, ph, wc) || !mbar_wait(v_full + st, (j / kKVStages) & 1, wc)) break;
+                tc_fence_after();
+                issue_pv(0, j);
+                if (more) {
+                    // S_A(j+1) overwrites P_A(j): wait until P_A(j) V_j has completed
+                    if (!mbar_wait(k_full + st1, ((j + 1) / kKVStages) & 1, wc) || !mbar_wait(o_done, ph, wc)) break;
+                    tc_fence_after();
+                    issue_s(0, j + 1);
+                }
+                if (!mbar_wait(p_full + 1, ph, wc)) break;
+                tc_fence_after();
+                issue_pv(1, j);
                 mma_commit(kv_empty + st);
-                mma_commit(o_done);
-                if (j + 2 < n_kv) ok = issue_s(j + 2);
+                if (more) {
+                    if (!mbar_wait(o_done + 1, ph, wc)) break;
+                    tc_fence_after();
+                    issue_s(1, j + 1);
+                }
             }
         }
     } else if (seg_len > 0) {
-        const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;                          // query row inside the tile
+        const int x = (warp - 2) >> 2;                             // query tile of this warpgroup
+        const int quarter = warp & 3;                              // TMEM lanes 32*quarter ..
+        const int r = quarter * 32 + lane;                         // query row inside the tile
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t tS = tmem + x * 128 + lane_off;
+        const uint32_t tO = tmem + 256 + x * 128 + lane_off;
         const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
-        float m = -INFINITY, l = 0.f;
-        uint8_t *prow = sP + r * 128;
+        float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
-            if (!mbar_wait(s_full + (j & 1), (j >> 1) & 1, wc)) { ok = false; break; }
+            if (!mbar_wait(s_full + x, j & 1, wc)) { ok = false; break; }
             tc_fence_after();
             uint32_t sr[128];
-            tmem_ld32(tS + (j & 1) * 128 + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(sr + 0));
-            tmem_ld32(tS + (j & 1) * 128 + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-            tmem_ld32(tS + (j & 1) * 128 + lane_off + 64, *reinterpret_cast<uint32_t(*)[32]>(sr + 64));
-            tmem_ld32(tS + (j & 1) * 128 + lane_off + 96, *reinterpret_cast<uint32_t(*)[32]>(sr + 96));
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * c));
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 4; ++c) reg_fence32(sr + 32 * c);
             const int kv_valid = min(kBKV, seg_len - j * kBKV);
-            float x[128];
-            float mx = -INFINITY;
+            if (kv_valid < kBKV) {   // last tile of the segment: keys past its end do not exist
 #pragma unroll
-            for (int k = 0; k < 128; ++k) {
-                x[k] = (k < kv_valid) ? __uint_as_float(sr[k]) * scale_log2 : -INFINITY;
-                mx = fmaxf(mx, x[k]);
+                for (int k = 0; k < 128; ++k)
+                    if (k >= kv_valid) sr[k] = __float_as_uint(-INFINITY);
             }
-            const float m_new = fmaxf(m, mx);
-            const float alpha = ex2(m - m_new);
-            float rs = 0.f;
+            // row max as a tree (independent partial maxima keep the pipes busy)
+            float m8[8];
 #pragma unroll
-            for (int k = 0; k < 128; ++k) {
-                x[k] = ex2(x[k] - m_new);
-                rs += x[k];
-            }
-            l = l * alpha + rs;
-            if (j > 0) {
-                if (!mbar_wait(o_done, (j - 1) & 1, wc)) { ok = false; break; }
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha < 1.0f)) {
+            for (int i = 0; i < 8; ++i) m8[i] = __uint_as_float(sr[i]);
 #pragma unroll
-                    for (int c = 0; c < 5; ++c) {
-                        uint32_t o[16];
-                        tmem_ld16(tO + lane_off + c * 16, o);
-                        tmem_wait_ld();
-                        reg_fence16(o);
+            for (int k = 8; k < 128; k += 8)
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st16(tO + lane_off + c * 16, o);
-                    }
-                    tmem_wait_st();
+                for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], __uint_as_float(sr[k + i]));
+            float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            mx *= scale_log2;
+            // O_x holds the sum through P_x(j-1) V_(j-1) here: S_x(j) was issued after it completed
+            const bool need = mx > m_used + kRescaleThreshold;
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+                const float alpha = need ? ex2(m_used - mx) : 1.0f;
+                l *= alpha;
+#pragma unroll
+                for (int c = 0; c < 5; ++c) {
+                    uint32_t o[16];
+                    tmem_ld16(tO + c * 16, o);
+                    tmem_wait_ld();
+                    reg_fence16(o);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st16(tO + c * 16, o);
                 }
+                tmem_wait_st();
             }
-            // P row r as bf16 into the 128B-swizzled, K-major tile: 16-byte chunk c of the
-            // 64-key atom goes to chunk c ^ (r % 8)
+            if (need) m_used = mx;
+            const float neg_m = -m_used;
+            float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[64];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const int atom = c >> 3, ch = c & 7;
-                uint4 v = make_uint4(pack_bf16x2(x[8 * c], x[8 * c + 1]), pack_bf16x2(x[8 * c + 2], x[8 * c + 3]),
-                                     pack_bf16x2(x[8 * c + 4], x[8 * c + 5]), pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
-                *reinterpret_cast<uint4 *>(prow + atom * 16384 + ((ch ^ (r & 7)) << 4)) = v;
+            for (int k = 0; k < 128; k += 2) {
+                const float p0 = ex2(fmaf(__uint_as_float(sr[k]), scale_log2, neg_m));
+                const float p1 = ex2(fmaf(__uint_as_float(sr[k + 1]), scale_log2, neg_m));
+                r8[(k >> 1) & 7] += p0 + p1;
+                pk[k >> 1] = pack_bf16x2(p0, p1);
             }
-            fence_proxy_async_smem();
+            const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+            l += rs;
+            tmem_st32(tS, pk);
+            tmem_st32(tS + 32, pk + 32);
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(p_full);
-            m = m_new;
+            mbar_arrive(p_full + x);
         }
-        if (ok && mbar_wait(o_done, (n_kv - 1) & 1, wc)) {
+        if (ok && mbar_wait(o_done + x, (n_kv - 1) & 1, wc)) {
             tc_fence_after();
             uint32_t o[80];
 #pragma unroll
-            for (int c = 0; c < 5; ++c) tmem_ld16(tO + lane_off + c * 16, o + c * 16);
+            for (int c = 0; c < 5; ++c) tmem_ld16(tO + c * 16, o + c * 16);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 5; ++c) reg_fence16(o + c * 16);
-            const int n_q = min(kBQ, seg_len - qt * kBQ);
-            if (r < n_q) {
+            const int row = pair * kQTilesPerCta * kBQ + x * kBQ + r;   // row inside the segment
+            if (row < seg_len) {
                 const float inv = 1.0f / l;
-                uint4 *dst = reinterpret_cast<uint4 *>(out + static_cast<int64_t>(q0 + r) * VIT_WIDTH + head * kD);
+                uint4 *dst = reinterpret_cast<uint4 *>(out + static_cast<int64_t>(seg_start + row) * VIT_WIDTH + head * kD);
 #pragma unroll
                 for (int q = 0; q < 10; ++q)
                     dst[q] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * q]) * inv, __uint_as_float(o[8 * q + 1]) * inv),
@@ -293,7 +324,7 @@ int attn_launch(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, v
         while (pos < order.size()) {
             const int sg = order[pos];
             const int len = cu_seqlens[sg + 1] - cu_seqlens[sg];
-            const int tiles = (len + vitk::kBQ - 1) / vitk::kBQ;
+            const int tiles = (len + vitk::kBQ * vitk::kQTilesPerCta - 1) / (vitk::kBQ * vitk::kQTilesPerCta);
             if (plan->n_seg == vitk::kMaxSegPerLaunch || plan->n_work + tiles > vitk::kMaxWorkPerLaunch) {
                 if (plan->n_seg == 0) return VIT_ERR_LIMIT;   // one segment alone exceeds a launch
                 break;
@@ -341,7 +372,7 @@ int attn_launch_stack(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_
         while (pos < n_seg) {
             const int sg = order[pos];
             const int len = cu_seqlens[sg + 1] - cu_seqlens[sg];
-            const int tiles = (len + vitk::kBQ - 1) / vitk::kBQ;
+            const int tiles = (len + vitk::kBQ * vitk::kQTilesPerCta - 1) / (vitk::kBQ * vitk::kQTilesPerCta);
             if (plan.n_seg == vitk::kMaxSegPerLaunch || plan.n_work + tiles > vitk::kMaxWorkPerLaunch) {
                 if (plan.n_seg == 0) return VIT_ERR_LIMIT;
                 break;
