@@ -227,10 +227,16 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
     VIT_TRY(vith::gemm_make_a_map(&mH4, h->H, M4, VIT_MERGE_DIM));
     VIT_TRY(vith::gemm_make_a_map(&mF4, h->F, M4, VIT_MERGE_DIM));
     VIT_TRY(vith::attn_make_map(&mQKV, h->QKV, P));
+    CUtensorMap cX, cQKV, cF, cF4, cOut;
+    VIT_TRY(vith::gemm_make_c_map(&cX, h->X, P, VIT_WIDTH, VIT_EPI_ADD_F32));
+    VIT_TRY(vith::gemm_make_c_map(&cQKV, h->QKV, P, 3 * VIT_WIDTH, VIT_EPI_QKV_ROPE));
+    VIT_TRY(vith::gemm_make_c_map(&cF, h->F, P, VIT_MLP, VIT_EPI_GELU_BF16));
+    VIT_TRY(vith::gemm_make_c_map(&cF4, h->F, M4, VIT_MERGE_DIM, VIT_EPI_GELU_BF16));
+    VIT_TRY(vith::gemm_make_c_map(&cOut, out, M4, d.out_dim, VIT_EPI_STORE_BF16));
 
     {
         ProfScope ps(h, s, P_PE);
-        VIT_TRY(vith::gemm_launch(mPatch, h->pe_map, h->X, d.pe_b, P, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32,
+        VIT_TRY(vith::gemm_launch(mPatch, h->pe_map, cX, d.pe_b, P, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32,
                                   nullptr, nullptr, h->status, s));
         ++nl;
     }
@@ -244,7 +250,7 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
         }
         {
             ProfScope ps(h, s, P_QKV);
-            VIT_TRY(vith::gemm_launch(mH, lm.qkv, h->QKV, L.qkv_b, P, 3 * VIT_WIDTH, VIT_WIDTH, VIT_EPI_QKV_ROPE,
+            VIT_TRY(vith::gemm_launch(mH, lm.qkv, cQKV, L.qkv_b, P, 3 * VIT_WIDTH, VIT_WIDTH, VIT_EPI_QKV_ROPE,
                                       h->pos, h->rope_cs, h->status, s));
             ++nl;
         }
@@ -255,7 +261,7 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
         }
         {
             ProfScope ps(h, s, P_PROJ);
-            VIT_TRY(vith::gemm_launch(mH, lm.proj, h->X, L.proj_b, P, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32, nullptr,
+            VIT_TRY(vith::gemm_launch(mH, lm.proj, cX, L.proj_b, P, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32, nullptr,
                                       nullptr, h->status, s));
             ++nl;
         }
@@ -266,13 +272,13 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
         }
         {
             ProfScope ps(h, s, P_FC1);
-            VIT_TRY(vith::gemm_launch(mH, lm.fc1, h->F, L.fc1_b, P, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16, nullptr,
+            VIT_TRY(vith::gemm_launch(mH, lm.fc1, cF, L.fc1_b, P, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16, nullptr,
                                       nullptr, h->status, s));
             ++nl;
         }
         {
             ProfScope ps(h, s, P_FC2);
-            VIT_TRY(vith::gemm_launch(mF, lm.fc2, h->X, L.fc2_b, P, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32, nullptr,
+            VIT_TRY(vith::gemm_launch(mF, lm.fc2, cX, L.fc2_b, P, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32, nullptr,
                                       nullptr, h->status, s));
             ++nl;
         }
@@ -285,13 +291,13 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
     }
     {
         ProfScope ps(h, s, P_M0);
-        VIT_TRY(vith::gemm_launch(mH4, h->m0_map, h->F, d.m0_b, M4, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16,
+        VIT_TRY(vith::gemm_launch(mH4, h->m0_map, cF4, d.m0_b, M4, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16,
                                   nullptr, nullptr, h->status, s));
         ++nl;
     }
     {
         ProfScope ps(h, s, P_M2);
-        VIT_TRY(vith::gemm_launch(mF4, h->m2_map, out, d.m2_b, M4, d.out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16,
+        VIT_TRY(vith::gemm_launch(mF4, h->m2_map, cOut, d.m2_b, M4, d.out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16,
                                   nullptr, nullptr, h->status, s));
         ++nl;
     }
@@ -483,11 +489,12 @@ int vit_op_gemm(const void *A, const void *B, const void *bias, void *C, int64_t
     if (epilogue == VIT_EPI_QKV_ROPE && (N != 3 * VIT_WIDTH || !pos || !rope_cs)) return VIT_ERR_ARG;
     if (M > (int64_t(1) << 30)) return VIT_ERR_LIMIT;
     if (!aligned16(A) || !aligned16(B) || !aligned16(C) || (bias && !aligned16(bias))) return VIT_ERR_ALIGN;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tc;
     int rc = vith::gemm_make_a_map(&ta, A, M, K);
     if (rc == VIT_OK) rc = vith::gemm_make_b_map(&tb, B, N, K, epilogue);
+    if (rc == VIT_OK) rc = vith::gemm_make_c_map(&tc, C, M, N, epilogue);
     if (rc != VIT_OK) return rc;
-    return vith::gemm_launch(ta, tb, C, bias, M, N, K, epilogue, pos, rope_cs, dev_status,
+    return vith::gemm_launch(ta, tb, tc, bias, M, N, K, epilogue, pos, rope_cs, dev_status,
                              static_cast<cudaStream_t>(stream));
 }
 

@@ -9,7 +9,9 @@
 //   warp 1      MMA issuer (one thread): tcgen05.mma 128xBNx16 into a TMEM accumulator;
 //               two accumulators so the epilogue of tile i overlaps the mainloop of tile i+1
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (one row per thread), bias,
-//               GELU / 2-D rope / residual add, stores to global memory
+//               GELU / 2-D rope, then the tile leaves through a double-buffered swizzled shared
+//               staging chunk and a TMA store -- or a TMA reduce-add into the fp32 residual
+//               stream, so the residual update never reads the residual into the SM.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -20,6 +22,7 @@ namespace vitk {
 constexpr int kBM = 128;
 constexpr int kBK = 64;           // 64 bf16 = 128 bytes: one 128B swizzle atom per row
 constexpr int kGemmThreads = 192;
+constexpr int kEpiBarrier = 1;    // named barrier of the 128 epilogue threads
 
 template <int BN>
 struct GemmShape {
@@ -28,12 +31,15 @@ struct GemmShape {
     static constexpr int B_BYTES = BN * kBK * 2;
     static constexpr int ACC_STRIDE = 256;    // TMEM columns between the two accumulators
     static constexpr int TMEM_COLS = 512;
-    static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + 256;
+    // output staging chunk: 128 rows x 128 bytes (32 fp32 or 64 bf16 columns), or for QKV one
+    // 80-wide head as five 128 x 32-byte boxes
+    static constexpr int STG_BYTES = BN == 240 ? 5 * 4096 : 16384;
+    static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + 2 * STG_BYTES + 256;
     static_assert(B_BYTES % 1024 == 0, "B stage must keep 1024-byte alignment");
+    static_assert(SMEM <= 232448, "shared memory per block");
 };
 
 struct GemmParams {
-    void *C;
     const __nv_bfloat16 *bias;
     const int32_t *pos;
     const float2 *rope_cs;
@@ -44,99 +50,58 @@ struct GemmParams {
 
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 
-// bias[col0 .. col0+n) -> v (n = 16 or 32; col0 a multiple of 16, bias 16-byte aligned)
+// v[0..NV) += bias[col0 ..] (bias 16-byte aligned, col0 a multiple of 8), columns >= N skipped
 template <int NV>
-__device__ __forceinline__ void add_bias(float *v, const __nv_bfloat16 *bias, int col0) {
+__device__ __forceinline__ void add_bias(float *v, const __nv_bfloat16 *bias, int col0, int N) {
     if (bias == nullptr) return;
-    const uint4 *b4 = reinterpret_cast<const uint4 *>(bias + col0);
 #pragma unroll
     for (int q = 0; q < NV / 8; ++q) {
-        uint4 u = __ldg(b4 + q);
-        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        if (col0 + 8 * q < N) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(bias + col0) + q);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            v[q * 8 + 2 * j] += bf16_lo(w[j]);
-            v[q * 8 + 2 * j + 1] += bf16_hi(w[j]);
-        }
-    }
-}
-
-template <int EPI>
-__device__ __forceinline__ void store_chunk32(const GemmParams &p, int row, int col0, float *v) {
-    if (EPI == VIT_EPI_STORE_F32 || EPI == VIT_EPI_ADD_F32) {
-        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.C) + static_cast<int64_t>(row) * p.N + col0);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            float4 o = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-            if (EPI == VIT_EPI_ADD_F32) {
-                float4 x = dst[q];
-                o.x += x.x; o.y += x.y; o.z += x.z; o.w += x.w;
+            for (int j = 0; j < 4; ++j) {
+                v[q * 8 + 2 * j] += bf16_lo(w[j]);
+                v[q * 8 + 2 * j + 1] += bf16_hi(w[j]);
             }
-            dst[q] = o;
-        }
-    } else {
-        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.C) + static_cast<int64_t>(row) * p.N + col0);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float a[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) a[j] = (EPI == VIT_EPI_GELU_BF16) ? gelu_erf(v[8 * q + j]) : v[8 * q + j];
-            dst[q] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
-                                pack_bf16x2(a[6], a[7]));
         }
     }
 }
 
-// columns col0 .. N-1 of a chunk that runs past N (N % 16 == 0, so 16 of the 32 are valid);
-// the loop bound is a compile-time constant so that v stays in registers
-template <int EPI>
-__device__ __forceinline__ void store_partial(const GemmParams &p, int row, int col0, const float *v, int n_valid) {
+// Writes one thread's row r of 128 bytes (eight 16-byte pieces) into a 128B-swizzled staging
+// chunk: piece q lands at piece q ^ (r % 8), the layout a SWIZZLE_128B TMA box expects.
+__device__ __forceinline__ void stage_row128(uint8_t *stg, int r, const uint32_t *w) {
+    uint8_t *row = stg + r * 128;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        if (j < n_valid) {
-            float x = v[j];
-            if (p.bias) x += __bfloat162float(p.bias[col0 + j]);
-            const int64_t o = static_cast<int64_t>(row) * p.N + col0 + j;
-            if (EPI == VIT_EPI_STORE_F32) static_cast<float *>(p.C)[o] = x;
-            else if (EPI == VIT_EPI_ADD_F32) static_cast<float *>(p.C)[o] += x;
-            else if (EPI == VIT_EPI_GELU_BF16) static_cast<__nv_bfloat16 *>(p.C)[o] = __float2bfloat16_rn(gelu_erf(x));
-            else static_cast<__nv_bfloat16 *>(p.C)[o] = __float2bfloat16_rn(x);
-        }
-    }
+    for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<uint4 *>(row + ((q ^ (r & 7)) << 4)) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
 }
 
-// One 80-wide head of the QKV output: bias, then the 2-D rope on q and k heads (columns < 2560).
-// Pair (d, d+40) turns by the angle of dim d: row position h for d < 20, column w for d >= 20.
-__device__ __forceinline__ void qkv_head(const GemmParams &p, int row, int col0, float *v) {
-    add_bias<80>(v, p.bias, col0);
-    if (col0 < 2 * VIT_WIDTH) {
-        const int hw = p.pos[row];
-        const float2 *ch = p.rope_cs + (hw >> 16) * 20;
-        const float2 *cw = p.rope_cs + (hw & 0xFFFF) * 20;
+// The 2-D rope on one 80-wide q or k head held in registers: pair (d, d+40) turns by the angle
+// of dim d, row position h for d < 20, column w for d >= 20.
+__device__ __forceinline__ void rope_head(float *v, int hw, const float2 *cs) {
+    const float2 *ch = cs + (hw >> 16) * 20;
+    const float2 *cw = cs + (hw & 0xFFFF) * 20;
 #pragma unroll
-        for (int d = 0; d < 40; ++d) {
-            const float2 cs = __ldg(d < 20 ? ch + d : cw + (d - 20));
-            const float x0 = v[d], x1 = v[d + 40];
-            v[d] = x0 * cs.x - x1 * cs.y;
-            v[d + 40] = x1 * cs.x + x0 * cs.y;
-        }
+    for (int d = 0; d < 40; ++d) {
+        const float2 c = __ldg(d < 20 ? ch + d : cw + (d - 20));
+        const float x0 = v[d], x1 = v[d + 40];
+        v[d] = x0 * c.x - x1 * c.y;
+        v[d + 40] = x1 * c.x + x0 * c.y;
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.C) + static_cast<int64_t>(row) * p.N + col0);
-#pragma unroll
-    for (int q = 0; q < 10; ++q)
-        dst[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                            pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
 }
 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb, GemmParams p) {
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
+                   const __grid_constant__ CUtensorMap tmc, GemmParams p) {
     using S = GemmShape<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + S::STAGES * S::A_BYTES;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sB + S::STAGES * S::B_BYTES);
+    uint8_t *sStg = sB + S::STAGES * S::B_BYTES;            // [2][STG_BYTES], 1024-aligned
+    uint64_t *full = reinterpret_cast<uint64_t *>(sStg + 2 * S::STG_BYTES);
     uint64_t *empty = full + S::STAGES;
     uint64_t *tfull = empty + S::STAGES;
     uint64_t *tempty = tfull + 2;
@@ -219,6 +184,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         const int quarter = warp & 3;   // TMEM lanes [32*quarter, 32*quarter+32) belong to this warp
+        const int r = quarter * 32 + lane;                      // row inside the tile
+        const bool leader = threadIdx.x == 64;                  // issues the TMA stores
+        int sc = 0;                                             // staging chunks used so far
+        // Before filling staging buffer sc % 2, the store that last read it must be done.
+        auto stage_acquire = [&]() {
+            if (leader && sc >= 2) bulk_wait_read<1>();
+            named_bar_sync(kEpiBarrier, 128);
+            return sStg + (sc & 1) * S::STG_BYTES;
+        };
+        auto stage_publish = [&]() {
+            fence_proxy_async_smem();
+            named_bar_sync(kEpiBarrier, 128);
+        };
         int local = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
             const int acc = local & 1;
@@ -226,46 +204,118 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!mbar_wait(tfull + acc, acc_phase, wc)) break;
             tc_fence_after();
             const int m0 = (tile / p.n_tiles) * kBM, n0 = (tile % p.n_tiles) * BN;
-            const int row = m0 + quarter * 32 + lane;
             const uint32_t t0 = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * S::ACC_STRIDE;
             if (EPI == VIT_EPI_QKV_ROPE) {
 #pragma unroll 1
                 for (int hh = 0; hh < BN / 80; ++hh) {
-                    uint32_t r[80];
+                    uint32_t u[80];
 #pragma unroll
-                    for (int c = 0; c < 5; ++c) tmem_ld16(t0 + hh * 80 + c * 16, r + c * 16);
+                    for (int c = 0; c < 5; ++c) tmem_ld16(t0 + hh * 80 + c * 16, u + c * 16);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 5; ++c) reg_fence16(r + c * 16);
+                    for (int c = 0; c < 5; ++c) reg_fence16(u + c * 16);
+                    if (hh == BN / 80 - 1) {   // accumulator fully read: hand it back to the MMA warp
+                        tc_fence_before();
+                        mbar_arrive(tempty + acc);
+                    }
                     float v[80];
 #pragma unroll
-                    for (int j = 0; j < 80; ++j) v[j] = __uint_as_float(r[j]);
-                    if (row < p.M) qkv_head(p, row, n0 + hh * 80, v);
+                    for (int j = 0; j < 80; ++j) v[j] = __uint_as_float(u[j]);
+                    const int col0 = n0 + hh * 80;
+                    add_bias<80>(v, p.bias, col0, p.N);
+                    const int row = m0 + r;
+                    if (col0 < 2 * VIT_WIDTH) rope_head(v, row < p.M ? p.pos[row] : 0, p.rope_cs);
+                    uint8_t *stg = stage_acquire();
+                    // five 32-byte-swizzled boxes of 16 columns: the 16-byte half h of row r goes
+                    // to half h ^ ((r >> 2) & 1)
+#pragma unroll
+                    for (int c = 0; c < 5; ++c) {
+                        uint8_t *rowp = stg + c * 4096 + r * 32;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const float *x = v + 16 * c + 8 * h;
+                            *reinterpret_cast<uint4 *>(rowp + ((h ^ ((r >> 2) & 1)) << 4)) =
+                                make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                                           pack_bf16x2(x[6], x[7]));
+                        }
+                    }
+                    stage_publish();
+                    if (leader) {
+#pragma unroll
+                        for (int c = 0; c < 5; ++c) tma_store_2d(&tmc, stg + c * 4096, col0 + 16 * c, m0);
+                        bulk_commit();
+                    }
+                    ++sc;
+                }
+            } else if (EPI == VIT_EPI_STORE_F32 || EPI == VIT_EPI_ADD_F32) {
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {     // 32 fp32 columns = one 128-byte row per chunk
+                    uint32_t u[32];
+                    tmem_ld32(t0 + c * 32, u);
+                    tmem_wait_ld();
+                    reg_fence32(u);
+                    if (c == BN / 32 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(tempty + acc);
+                    }
+                    const int col0 = n0 + c * 32;
+                    if (col0 < p.N) {                   // uniform across the CTA
+                        float v[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(u[j]);
+                        add_bias<32>(v, p.bias, col0, p.N);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(v[j]);
+                        uint8_t *stg = stage_acquire();
+                        stage_row128(stg, r, u);
+                        stage_publish();
+                        if (leader) {
+                            if (EPI == VIT_EPI_ADD_F32) tma_reduce_add_2d(&tmc, stg, col0, m0);
+                            else tma_store_2d(&tmc, stg, col0, m0);
+                            bulk_commit();
+                        }
+                        ++sc;
+                    }
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(t0 + c * 32, r);
+                for (int c = 0; c < BN / 64; ++c) {     // 64 bf16 columns = one 128-byte row per chunk
+                    uint32_t u[64];
+                    tmem_ld32(t0 + c * 64, *reinterpret_cast<uint32_t(*)[32]>(u));
+                    tmem_ld32(t0 + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
                     tmem_wait_ld();
-                    reg_fence32(r);
-                    const int col0 = n0 + c * 32;
-                    if (row < p.M && col0 < p.N) {
-                        float v[32];
+                    reg_fence32(u);
+                    reg_fence32(u + 32);
+                    if (c == BN / 64 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(tempty + acc);
+                    }
+                    const int col0 = n0 + c * 64;
+                    if (col0 < p.N) {
+                        float v[64];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-                        if (col0 + 32 <= p.N) {
-                            add_bias<32>(v, p.bias, col0);
-                            store_chunk32<EPI>(p, row, col0, v);
-                        } else {
-                            store_partial<EPI>(p, row, col0, v, p.N - col0);
+                        for (int j = 0; j < 64; ++j) v[j] = __uint_as_float(u[j]);
+                        add_bias<64>(v, p.bias, col0, p.N);
+                        uint32_t w[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            float a = v[2 * j], b = v[2 * j + 1];
+                            if (EPI == VIT_EPI_GELU_BF16) { a = gelu_erf(a); b = gelu_erf(b); }
+                            w[j] = pack_bf16x2(a, b);
                         }
+                        uint8_t *stg = stage_acquire();
+                        stage_row128(stg, r, w);
+                        stage_publish();
+                        if (leader) {
+                            tma_store_2d(&tmc, stg, col0, m0);
+                            bulk_commit();
+                        }
+                        ++sc;
                     }
                 }
             }
-            tc_fence_before();
-            mbar_arrive(tempty + acc);
         }
+        if (leader) bulk_wait<0>();             // every store has landed before the CTA exits
     }
 
     tc_fence_before();
@@ -292,8 +342,24 @@ int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue)
                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+int gemm_make_c_map(CUtensorMap *map, void *C, int64_t M, int N, int epilogue) {
+    switch (epilogue) {
+        case VIT_EPI_STORE_F32:
+        case VIT_EPI_ADD_F32:
+            return tmap_2d(map, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, M, static_cast<uint64_t>(N) * 4, 32,
+                           vitk::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+        case VIT_EPI_QKV_ROPE:
+            return tmap_2d(map, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, static_cast<uint64_t>(N) * 2, 16,
+                           vitk::kBM, CU_TENSOR_MAP_SWIZZLE_32B);
+        default:
+            return tmap_2d(map, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, static_cast<uint64_t>(N) * 2, 64,
+                           vitk::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+}
+
 template <int BN, int EPI>
-static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const vitk::GemmParams &p, cudaStream_t s) {
+static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc, const vitk::GemmParams &p,
+                      cudaStream_t s) {
     using S = vitk::GemmShape<BN>;
     static bool configured[64] = {};   // the attribute is set once per device
     int dev = 0;
@@ -307,15 +373,15 @@ static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const vitk::
     const int total = p.m_tiles * p.n_tiles;
     const int sms = device_sm_count();
     const int grid = total < sms ? total : sms;
-    vitk::gemm_tc_kernel<BN, EPI><<<grid, vitk::kGemmThreads, S::SMEM, s>>>(ta, tb, p);
+    vitk::gemm_tc_kernel<BN, EPI><<<grid, vitk::kGemmThreads, S::SMEM, s>>>(ta, tb, tc, p);
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 
-int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, void *C, const void *bias, int64_t M, int N, int K,
-                int epilogue, const int32_t *pos, const float *rope_cs, int32_t *status, cudaStream_t s) {
+int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc, const void *bias, int64_t M,
+                int N, int K, int epilogue, const int32_t *pos, const float *rope_cs, int32_t *status,
+                cudaStream_t s) {
     if (M <= 0) return VIT_OK;
     vitk::GemmParams p{};
-    p.C = C;
     p.bias = static_cast<const __nv_bfloat16 *>(bias);
     p.pos = pos;
     p.rope_cs = reinterpret_cast<const float2 *>(rope_cs);
@@ -328,19 +394,19 @@ int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, void *C, const voi
     switch (epilogue) {
         case VIT_EPI_QKV_ROPE:
             p.n_tiles = N / 240;
-            return launch_one<240, VIT_EPI_QKV_ROPE>(ta, tb, p, s);
+            return launch_one<240, VIT_EPI_QKV_ROPE>(ta, tb, tc, p, s);
         case VIT_EPI_STORE_F32:
             p.n_tiles = (N + 255) / 256;
-            return launch_one<256, VIT_EPI_STORE_F32>(ta, tb, p, s);
+            return launch_one<256, VIT_EPI_STORE_F32>(ta, tb, tc, p, s);
         case VIT_EPI_ADD_F32:
             p.n_tiles = (N + 255) / 256;
-            return launch_one<256, VIT_EPI_ADD_F32>(ta, tb, p, s);
+            return launch_one<256, VIT_EPI_ADD_F32>(ta, tb, tc, p, s);
         case VIT_EPI_STORE_BF16:
             p.n_tiles = (N + 255) / 256;
-            return launch_one<256, VIT_EPI_STORE_BF16>(ta, tb, p, s);
+            return launch_one<256, VIT_EPI_STORE_BF16>(ta, tb, tc, p, s);
         case VIT_EPI_GELU_BF16:
             p.n_tiles = (N + 255) / 256;
-            return launch_one<256, VIT_EPI_GELU_BF16>(ta, tb, p, s);
+            return launch_one<256, VIT_EPI_GELU_BF16>(ta, tb, tc, p, s);
         default:
             return VIT_ERR_ARG;
     }

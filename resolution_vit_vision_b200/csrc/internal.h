@@ -20,8 +20,11 @@ int check_device();   // VIT_OK when the current device is sm_100
 // ---- GEMM (gemm.cu). A bf16 [M, K], B bf16 [N, K]. The B map may be prebuilt (weights).
 int gemm_make_a_map(CUtensorMap *map, const void *A, int64_t M, int K);
 int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue);
-int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, void *C, const void *bias, int64_t M, int N, int K,
-                int epilogue, const int32_t *pos, const float *rope_cs, int32_t *status, cudaStream_t s);
+// C [M, N]: fp32 for STORE_F32 / ADD_F32 (the output is written, or added, by TMA), else bf16
+int gemm_make_c_map(CUtensorMap *map, void *C, int64_t M, int N, int epilogue);
+int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc, const void *bias, int64_t M,
+                int N, int K, int epilogue, const int32_t *pos, const float *rope_cs, int32_t *status,
+                cudaStream_t s);
 
 // ---- attention (attention.cu). qkv bf16 [P, 3840].
 int attn_make_map(CUtensorMap *map, const void *qkv, int64_t P);

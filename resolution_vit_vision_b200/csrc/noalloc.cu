@@ -100,28 +100,34 @@ extern "C" int vit_encode_noalloc(const void *patches, const int32_t *grid_thw, 
     NA_TRY(vith::gemm_make_a_map(&mH4, H, M4, VIT_MERGE_DIM));
     NA_TRY(vith::gemm_make_a_map(&mF4, F, M4, VIT_MERGE_DIM));
     NA_TRY(vith::attn_make_map(&mQKV, QKV, P));
-    NA_TRY(vith::gemm_launch(mPatch, h->pe_map, X, d.pe_b, P, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32, nullptr,
+    CUtensorMap cX, cQKV, cF, cF4, cOut;
+    NA_TRY(vith::gemm_make_c_map(&cX, X, P, VIT_WIDTH, VIT_EPI_ADD_F32));
+    NA_TRY(vith::gemm_make_c_map(&cQKV, QKV, P, 3 * VIT_WIDTH, VIT_EPI_QKV_ROPE));
+    NA_TRY(vith::gemm_make_c_map(&cF, F, P, VIT_MLP, VIT_EPI_GELU_BF16));
+    NA_TRY(vith::gemm_make_c_map(&cF4, F, M4, VIT_MERGE_DIM, VIT_EPI_GELU_BF16));
+    NA_TRY(vith::gemm_make_c_map(&cOut, out, M4, d.out_dim, VIT_EPI_STORE_BF16));
+    NA_TRY(vith::gemm_launch(mPatch, h->pe_map, cX, d.pe_b, P, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32, nullptr,
                              nullptr, dev_status, s));
     for (int l = 0; l < d.depth; ++l) {
         const vit_layer_w &L = h->layers[l];
         const vith::LayerMaps &lm = h->maps[l];
         NA_TRY(vith::layernorm_launch(X, L.ln1_w, L.ln1_b, H, P, d.ln_eps, nullptr, s));
-        NA_TRY(vith::gemm_launch(mH, lm.qkv, QKV, L.qkv_b, P, 3 * VIT_WIDTH, VIT_WIDTH, VIT_EPI_QKV_ROPE, pos,
+        NA_TRY(vith::gemm_launch(mH, lm.qkv, cQKV, L.qkv_b, P, 3 * VIT_WIDTH, VIT_WIDTH, VIT_EPI_QKV_ROPE, pos,
                                  rope_cs, dev_status, s));
         NA_TRY(vith::attn_launch_stack(mQKV, cu, n_seg, H, dev_status, s));
-        NA_TRY(vith::gemm_launch(mH, lm.proj, X, L.proj_b, P, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32, nullptr, nullptr,
+        NA_TRY(vith::gemm_launch(mH, lm.proj, cX, L.proj_b, P, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32, nullptr, nullptr,
                                  dev_status, s));
         NA_TRY(vith::layernorm_launch(X, L.ln2_w, L.ln2_b, H, P, d.ln_eps, nullptr, s));
-        NA_TRY(vith::gemm_launch(mH, lm.fc1, F, L.fc1_b, P, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16, nullptr, nullptr,
+        NA_TRY(vith::gemm_launch(mH, lm.fc1, cF, L.fc1_b, P, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16, nullptr, nullptr,
                                  dev_status, s));
-        NA_TRY(vith::gemm_launch(mF, lm.fc2, X, L.fc2_b, P, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32, nullptr, nullptr,
+        NA_TRY(vith::gemm_launch(mF, lm.fc2, cX, L.fc2_b, P, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32, nullptr, nullptr,
                                  dev_status, s));
         h->launches += 7;
     }
     NA_TRY(vith::layernorm_launch(X, d.lnq_w, d.lnq_b, H, P, d.ln_eps, d.patch_order == 1 ? merge_row : nullptr, s));
-    NA_TRY(vith::gemm_launch(mH4, h->m0_map, F, d.m0_b, M4, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16, nullptr,
+    NA_TRY(vith::gemm_launch(mH4, h->m0_map, cF4, d.m0_b, M4, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16, nullptr,
                              nullptr, dev_status, s));
-    NA_TRY(vith::gemm_launch(mF4, h->m2_map, out, d.m2_b, M4, d.out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16, nullptr,
+    NA_TRY(vith::gemm_launch(mF4, h->m2_map, cOut, d.m2_b, M4, d.out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16, nullptr,
                              nullptr, dev_status, s));
     h->launches += 5;
     return VIT_OK;
