@@ -48,7 +48,23 @@ struct GemmParams {
     int m_tiles, n_tiles, k_blocks;
 };
 
-__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+// GELU(x) = x Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), with erf from Abramowitz & Stegun,
+// Handbook of Mathematical Functions, eq. 7.1.26 (Hastings' approximation): for z >= 0,
+// erfc(z) = t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2) + e(z), t = 1 / (1 + p z),
+// |e(z)| <= 1.5e-7. For x < 0, 1 + erf(x / sqrt 2) = erfc(|x| / sqrt 2) is taken directly from
+// that product, so large negative x keep their relative accuracy. Two MUFU operations (rcp, ex2)
+// and ten FMA-pipe operations per element.
+__device__ __forceinline__ float gelu_erf(float x) {
+    const float z = fabsf(x) * 0.70710678118654752f;
+    float t;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.3275911f, z, 1.0f)));
+    const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f), -0.284496736f),
+                                0.254829592f);
+    float e;   // exp(-z^2) = 2^(-z^2 log2 e)
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-z * z * 1.4426950408889634f));
+    const float erfc_z = poly * e;
+    return 0.5f * x * (x >= 0.f ? 2.0f - erfc_z : erfc_z);
+}
 
 // v[0..NV) += bias[col0 ..] (bias 16-byte aligned, col0 a multiple of 8), columns >= N skipped
 template <int NV>
