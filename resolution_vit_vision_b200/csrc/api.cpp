@@ -220,13 +220,14 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
         ++nl;
     }
 
-    CUtensorMap mPatch, mH, mF, mH4, mF4, mQKV;
+    CUtensorMap mPatch, mH, mF, mH4, mF4;
+    vith::AttnMaps mQKV;
     VIT_TRY(vith::gemm_make_a_map(&mPatch, patches, P, VIT_PATCH_DIM));
     VIT_TRY(vith::gemm_make_a_map(&mH, h->H, P, VIT_WIDTH));
     VIT_TRY(vith::gemm_make_a_map(&mF, h->F, P, VIT_MLP));
     VIT_TRY(vith::gemm_make_a_map(&mH4, h->H, M4, VIT_MERGE_DIM));
     VIT_TRY(vith::gemm_make_a_map(&mF4, h->F, M4, VIT_MERGE_DIM));
-    VIT_TRY(vith::attn_make_map(&mQKV, h->QKV, P));
+    VIT_TRY(vith::attn_make_maps(&mQKV, h->QKV, P));
     CUtensorMap cX, cQKV, cF, cF4, cOut;
     VIT_TRY(vith::gemm_make_c_map(&cX, h->X, P, VIT_WIDTH, VIT_EPI_ADD_F32));
     VIT_TRY(vith::gemm_make_c_map(&cQKV, h->QKV, P, 3 * VIT_WIDTH, VIT_EPI_QKV_ROPE));
@@ -528,8 +529,8 @@ int vit_op_attention(const void *qkv, int64_t P, const int32_t *cu_seqlens, int 
         if (cu_seqlens[i + 1] < cu_seqlens[i]) return VIT_ERR_ARG;
     if (P > VIT_MAX_PATCHES) return VIT_ERR_LIMIT;
     if (!aligned16(qkv) || !aligned16(out)) return VIT_ERR_ALIGN;
-    CUtensorMap t;
-    const int rc = vith::attn_make_map(&t, qkv, P);
+    vith::AttnMaps t;
+    const int rc = vith::attn_make_maps(&t, qkv, P);
     if (rc != VIT_OK) return rc;
     return vith::attn_launch(t, cu_seqlens, n_seg, out, dev_status, static_cast<cudaStream_t>(stream));
 }

@@ -25,17 +25,24 @@
 namespace vitk {
 
 constexpr int kAttnThreads = 320;                 // 10 warps
-constexpr int kBQ = 128, kBKV = 128, kD = 80;
+constexpr int kBQ = 128, kBKV = 112, kD = 80;     // query tile, key tile, head dim
 constexpr int kQTilesPerCta = 2;                  // query tiles A and B share every K/V tile
-constexpr int kKVStages = 3;
-constexpr int kTileBytes = kBQ * kD * 2;          // 20480: 5 boxes of 128 rows x 32 bytes
-constexpr int kBoxBytes = 128 * 32;               // one 16-column box
-constexpr int kAttnSmem = 1024 + kTileBytes * (kQTilesPerCta + 2 * kKVStages) + 256;
+constexpr int kKVStages = 4;
+constexpr int kQBytes = kBQ * kD * 2;             // 20480: 5 boxes of 128 rows x 32 bytes
+constexpr int kQBox = kBQ * 32;
+constexpr int kKVBytes = kBKV * kD * 2;           // 17920: 5 boxes of 112 rows x 32 bytes
+constexpr int kKVBox = kBKV * 32;
+constexpr int kAttnSmem = 1024 + kQBytes * kQTilesPerCta + kKVBytes * 2 * kKVStages + 256;
 constexpr int kMaxSegPerLaunch = 512;
 constexpr int kMaxWorkPerLaunch = 4096;
-// Lazy rescaling: the exponent offset of a row only moves when its running max grows by more
-// than this (log2 units), so P stays below 2^8 and O is rarely rescaled.
+// Lazy rescaling: a row's exponent offset only moves when its running max grows by more than
+// this (log2 units), so P stays below 2^8 and O is rarely rescaled.
 constexpr float kRescaleThreshold = 8.0f;
+// TMEM columns of query tile x: scores S_x (112), P_x (bf16 pairs, 56 used of 64), O_x (80).
+__host__ __device__ constexpr uint32_t col_s(int x) { return x * 112; }
+__host__ __device__ constexpr uint32_t col_p(int x) { return 224 + x * 64; }
+__host__ __device__ constexpr uint32_t col_o(int x) { return 352 + x * 80; }
+static_assert(col_o(1) + 80 <= 512, "TMEM budget");
 
 // Work list and segment starts travel as a kernel parameter (no device-side plan buffer).
 struct AttnPlan {
@@ -52,25 +59,28 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// TMEM columns: S_A / P_A at 0, S_B / P_B at 128 (P, bf16 pairs, overwrites the first 64 columns
-// of its S once the scores are in registers), O_A at 256, O_B at 384 (80 columns each).
+// Warp roles: 0 TMA producer, 1 MMA issuer, 2..5 softmax of query tile A, 6..9 of tile B (one
+// query row per thread). Each tile has its own score and P buffers, so S_x(j+1) = Q_x K_(j+1)^T
+// runs on the tensor core while the softmax warpgroup is still turning S_x(j) into P_x(j).
 // 10 warps put 3 warps on two of the SM's four sub-partitions (16K registers each), which caps
 // a thread at 168 registers.
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ AttnPlan plan,
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tkv,
+                   const __grid_constant__ AttnPlan plan,
                    __nv_bfloat16 *__restrict__ out, int32_t *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem;                                   // [2][5 boxes]
-    uint8_t *sK = sQ + kQTilesPerCta * kTileBytes;
-    uint8_t *sV = sK + kKVStages * kTileBytes;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kKVStages * kTileBytes);
+    uint8_t *sK = sQ + kQTilesPerCta * kQBytes;
+    uint8_t *sV = sK + kKVStages * kKVBytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kKVStages * kKVBytes);
     uint64_t *q_full = bars;
     uint64_t *k_full = bars + 1;
     uint64_t *v_full = k_full + kKVStages;
     uint64_t *kv_empty = v_full + kKVStages;
     uint64_t *s_full = kv_empty + kKVStages;     // [2] per query tile
-    uint64_t *p_full = s_full + 2;               // [2]
+    uint64_t *s_free = s_full + 2;               // [2]
+    uint64_t *p_full = s_free + 2;               // [2]
     uint64_t *o_done = p_full + 2;               // [2]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -92,6 +102,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(s_full + x, 1);
+            mbar_init(s_free + x, 128);
             mbar_init(p_full + x, 128);
             mbar_init(o_done + x, 1);
         }
@@ -111,21 +122,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (warp == 0) {
         if (lane == 0 && seg_len > 0) {
             tma_prefetch(&tm);
-            mbar_expect_tx(q_full, kQTilesPerCta * kTileBytes);
+            tma_prefetch(&tkv);
+            mbar_expect_tx(q_full, kQTilesPerCta * kQBytes);
             for (int x = 0; x < kQTilesPerCta; ++x)
                 for (int c = 0; c < 5; ++c)
-                    tma_load_2d(sQ + x * kTileBytes + c * kBoxBytes, &tm, q_full, head * kD + c * 16, q0 + x * kBQ);
+                    tma_load_2d(sQ + x * kQBytes + c * kQBox, &tm, q_full, head * kD + c * 16, q0 + x * kBQ);
             for (int j = 0; j < n_kv; ++j) {
                 const int st = j % kKVStages;
                 const uint32_t ph = (j / kKVStages) & 1;
                 if (!mbar_wait(kv_empty + st, ph ^ 1u, wc)) break;
                 const int r0 = seg_start + j * kBKV;
-                mbar_expect_tx(k_full + st, kTileBytes);
+                mbar_expect_tx(k_full + st, kKVBytes);
                 for (int c = 0; c < 5; ++c)
-                    tma_load_2d(sK + st * kTileBytes + c * kBoxBytes, &tm, k_full + st, VIT_WIDTH + head * kD + c * 16, r0);
-                mbar_expect_tx(v_full + st, kTileBytes);
+                    tma_load_2d(sK + st * kKVBytes + c * kKVBox, &tkv, k_full + st, VIT_WIDTH + head * kD + c * 16, r0);
+                mbar_expect_tx(v_full + st, kKVBytes);
                 for (int c = 0; c < 5; ++c)
-                    tma_load_2d(sV + st * kTileBytes + c * kBoxBytes, &tm, v_full + st,
+                    tma_load_2d(sV + st * kKVBytes + c * kKVBox, &tkv, v_full + st,
                                 2 * VIT_WIDTH + head * kD + c * 16, r0);
             }
         }
@@ -134,24 +146,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             constexpr uint32_t idS = idesc_bf16(kBQ, kBKV, false, false);
             constexpr uint32_t idO = idesc_bf16(kBQ, kD, false, true);   // V is N(=head dim)-major
             const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
-            // S_x(j) = Q_x K_j^T into TMEM columns 128 x
-            auto issue_s = [&](int x, int j) {
+            auto issue_s = [&](int x, int j) {    // S_x = Q_x K_j^T
                 const int st = j % kKVStages;
 #pragma unroll
                 for (int c = 0; c < 5; ++c) {
-                    const uint64_t da = smem_desc(qa + x * kTileBytes + c * kBoxBytes, 16, 256, kSwizzle32B);
-                    const uint64_t db = smem_desc(ka + st * kTileBytes + c * kBoxBytes, 16, 256, kSwizzle32B);
-                    mma_bf16_ss(tmem + x * 128, da, db, idS, c > 0 ? 1u : 0u);
+                    const uint64_t da = smem_desc(qa + x * kQBytes + c * kQBox, 16, 256, kSwizzle32B);
+                    const uint64_t db = smem_desc(ka + st * kKVBytes + c * kKVBox, 16, 256, kSwizzle32B);
+                    mma_bf16_ss(tmem + col_s(x), da, db, idS, c > 0 ? 1u : 0u);
                 }
                 mma_commit(s_full + x);
             };
-            // O_x += P_x(j) V_j, P_x read from TMEM (8 columns per 16 keys)
-            auto issue_pv = [&](int x, int j) {
+            auto issue_pv = [&](int x, int j) {   // O_x += P_x V_j, P_x read from TMEM (8 columns per 16 keys)
                 const int st = j % kKVStages;
 #pragma unroll
                 for (int kk = 0; kk < kBKV / 16; ++kk) {
-                    const uint64_t db = smem_desc(va + st * kTileBytes + kk * 512, 4096, 256, kSwizzle32B);
-                    mma_bf16_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
+                    const uint64_t db = smem_desc(va + st * kKVBytes + kk * 512, kKVBox, 256, kSwizzle32B);
+                    mma_bf16_ts(tmem + col_o(x), tmem + col_p(x) + kk * 8, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(o_done + x);
             };
@@ -164,26 +174,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int j = 0; ok && j < n_kv; ++j) {
                 const int st = j % kKVStages;
                 const uint32_t ph = j & 1;
-                const bool more = j + 1 < n_kv;
-                const int st1 = (j + 1) % kKVStages;
+                if (j + 1 < n_kv) {
+                    // the next scores as soon as each softmax warpgroup has read this step's
+                    const int st1 = (j + 1) % kKVStages;
+                    if (!mbar_wait(k_full + st1, ((j + 1) / kKVStages) & 1, wc) || !mbar_wait(s_free, ph, wc)) break;
+                    tc_fence_after();
+                    issue_s(0, j + 1);
+                    if (!mbar_wait(s_free + 1, ph, wc)) break;
+                    tc_fence_after();
+                    issue_s(1, j + 1);
+                }
                 if (!mbar_wait(p_full, ph, wc) || !mbar_wait(v_full + st, (j / kKVStages) & 1, wc)) break;
                 tc_fence_after();
                 issue_pv(0, j);
-                if (more) {
-                    // S_A(j+1) overwrites P_A(j): wait until P_A(j) V_j has completed
-                    if (!mbar_wait(k_full + st1, ((j + 1) / kKVStages) & 1, wc) || !mbar_wait(o_done, ph, wc)) break;
-                    tc_fence_after();
-                    issue_s(0, j + 1);
-                }
                 if (!mbar_wait(p_full + 1, ph, wc)) break;
                 tc_fence_after();
                 issue_pv(1, j);
                 mma_commit(kv_empty + st);
-                if (more) {
-                    if (!mbar_wait(o_done + 1, ph, wc)) break;
-                    tc_fence_after();
-                    issue_s(1, j + 1);
-                }
             }
         }
     } else if (seg_len > 0) {
@@ -191,37 +198,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int quarter = warp & 3;                              // TMEM lanes 32*quarter ..
         const int r = quarter * 32 + lane;                         // query row inside the tile
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint32_t tS = tmem + x * 128 + lane_off;
-        const uint32_t tO = tmem + 256 + x * 128 + lane_off;
+        const uint32_t tS = tmem + col_s(x) + lane_off;
+        const uint32_t tP = tmem + col_p(x) + lane_off;
+        const uint32_t tO = tmem + col_o(x) + lane_off;
         const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
             if (!mbar_wait(s_full + x, j & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            uint32_t sr[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * c));
+            uint32_t sr[112];
+            tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(sr));
+            tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+            tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(sr + 64));
+            tmem_ld16(tS + 96, sr + 96);
             tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) reg_fence32(sr + 32 * c);
+            reg_fence32(sr);
+            reg_fence32(sr + 32);
+            reg_fence32(sr + 64);
+            reg_fence16(sr + 96);
+            tc_fence_before();
+            mbar_arrive(s_free + x);                               // S_x may be overwritten now
             const int kv_valid = min(kBKV, seg_len - j * kBKV);
-            if (kv_valid < kBKV) {   // last tile of the segment: keys past its end do not exist
+            if (kv_valid < kBKV) {   // last key tile of the segment
 #pragma unroll
-                for (int k = 0; k < 128; ++k)
+                for (int k = 0; k < kBKV; ++k)
                     if (k >= kv_valid) sr[k] = __float_as_uint(-INFINITY);
             }
-            // row max as a tree (independent partial maxima keep the pipes busy)
             float m8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) m8[i] = __uint_as_float(sr[i]);
 #pragma unroll
-            for (int k = 8; k < 128; k += 8)
+            for (int k = 8; k < kBKV; k += 8)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], __uint_as_float(sr[k + i]));
-            float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-            mx *= scale_log2;
-            // O_x holds the sum through P_x(j-1) V_(j-1) here: S_x(j) was issued after it completed
+            const float mx =
+                fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
+                scale_log2;
+            // P_x(j-1) V_(j-1) must be complete before O_x is rescaled or P_x is overwritten
+            if (j > 0) {
+                if (!mbar_wait(o_done + x, (j - 1) & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+            }
             const bool need = mx > m_used + kRescaleThreshold;
             if (j > 0 && __any_sync(0xffffffffu, need)) {
                 const float alpha = need ? ex2(m_used - mx) : 1.0f;
@@ -241,18 +259,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (need) m_used = mx;
             const float neg_m = -m_used;
             float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[64];
 #pragma unroll
-            for (int k = 0; k < 128; k += 2) {
-                const float p0 = ex2(fmaf(__uint_as_float(sr[k]), scale_log2, neg_m));
-                const float p1 = ex2(fmaf(__uint_as_float(sr[k + 1]), scale_log2, neg_m));
-                r8[(k >> 1) & 7] += p0 + p1;
-                pk[k >> 1] = pack_bf16x2(p0, p1);
+            for (int half = 0; half < 2; ++half) {   // keys [0, 64) and [64, 112) (+ 16 zero pad)
+                uint32_t pk[32];
+#pragma unroll
+                for (int k = 0; k < 64; k += 2) {
+                    const int kk = 64 * half + k;
+                    float p0 = 0.f, p1 = 0.f;
+                    if (kk < kBKV) {
+                        p0 = ex2(fmaf(__uint_as_float(sr[kk]), scale_log2, neg_m));
+                        p1 = ex2(fmaf(__uint_as_float(sr[kk + 1]), scale_log2, neg_m));
+                    }
+                    r8[(k >> 1) & 7] += p0 + p1;
+                    pk[k >> 1] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(tP + 32 * half, pk);
             }
-            const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
-            l += rs;
-            tmem_st32(tS, pk);
-            tmem_st32(tS + 32, pk + 32);
+            l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(p_full + x);
@@ -292,14 +315,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 namespace vith {
 
-int attn_make_map(CUtensorMap *map, const void *qkv, int64_t P) {
-    return tmap_2d(map, qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * VIT_WIDTH, static_cast<uint64_t>(P),
-                   3 * VIT_WIDTH * 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
+// Two views of the [P, 3840] QKV buffer, 16-column boxes with 32-byte swizzle: query tiles of
+// 128 rows and key / value tiles of kBKV rows.
+int attn_make_maps(AttnMaps *m, const void *qkv, int64_t P) {
+    int rc = tmap_2d(&m->q, qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * VIT_WIDTH, static_cast<uint64_t>(P),
+                     3 * VIT_WIDTH * 2, 16, vitk::kBQ, CU_TENSOR_MAP_SWIZZLE_32B);
+    if (rc == VIT_OK)
+        rc = tmap_2d(&m->kv, qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * VIT_WIDTH, static_cast<uint64_t>(P),
+                     3 * VIT_WIDTH * 2, 16, vitk::kBKV, CU_TENSOR_MAP_SWIZZLE_32B);
+    return rc;
 }
 
 // cu_seqlens: HOST [n_seg + 1]. Builds the (segment, q-tile) list, longest segments first,
 // and launches as many kernels as the per-launch limits need.
-int attn_launch(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
+int attn_launch(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
                 cudaStream_t s) {
     static bool configured[64] = {};
     int dev = 0;
@@ -337,7 +366,7 @@ int attn_launch(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, v
         }
         if (plan->n_work > 0) {
             vitk::attn_tc_kernel<<<plan->n_work * VIT_HEADS, vitk::kAttnThreads, vitk::kAttnSmem, s>>>(
-                tqkv, *plan, static_cast<__nv_bfloat16 *>(out), status);
+                tqkv.q, tqkv.kv, *plan, static_cast<__nv_bfloat16 *>(out), status);
             if (cudaGetLastError() != cudaSuccess) return VIT_ERR_CUDA;
         }
     }
@@ -346,7 +375,7 @@ int attn_launch(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, v
 
 // attn_launch with the schedule kept on the host stack and an in-place sort (ties broken by
 // segment index, the order attn_launch's stable sort gives), for callers that must not allocate.
-int attn_launch_stack(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
+int attn_launch_stack(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
                       cudaStream_t s) {
     if (n_seg < 0 || n_seg > VIT_MAX_SEGMENTS) return VIT_ERR_LIMIT;
     static bool configured[64] = {};
@@ -385,7 +414,7 @@ int attn_launch_stack(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_
         }
         if (plan.n_work > 0) {
             vitk::attn_tc_kernel<<<plan.n_work * VIT_HEADS, vitk::kAttnThreads, vitk::kAttnSmem, s>>>(
-                tqkv, plan, static_cast<__nv_bfloat16 *>(out), status);
+                tqkv.q, tqkv.kv, plan, static_cast<__nv_bfloat16 *>(out), status);
             if (cudaGetLastError() != cudaSuccess) return VIT_ERR_CUDA;
         }
     }

@@ -27,9 +27,12 @@ int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap 
                 cudaStream_t s);
 
 // ---- attention (attention.cu). qkv bf16 [P, 3840].
-int attn_make_map(CUtensorMap *map, const void *qkv, int64_t P);
+struct AttnMaps {
+    CUtensorMap q, kv;
+};
+int attn_make_maps(AttnMaps *m, const void *qkv, int64_t P);
 // cu_seqlens: HOST [n_seg + 1]; the (segment, q-tile) work list is built here, longest first
-int attn_launch(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
+int attn_launch(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
                 cudaStream_t s);
 
 // ---- small kernels (misc.cu)
@@ -40,7 +43,7 @@ int rope_table_launch(float *cs, int n_pos, cudaStream_t s);
 int positions_launch(const int32_t *grid_thw, int n_images, int64_t P, int patch_order, int32_t *pos,
                      int32_t *merge_row, cudaStream_t s);
 // the same launches with their host-side tables on the stack (no heap use)
-int attn_launch_stack(const CUtensorMap &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
+int attn_launch_stack(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
                       cudaStream_t s);
 int positions_launch_stack(const int32_t *grid_thw, int n_images, int64_t P, int patch_order, int32_t *pos,
                            int32_t *merge_row, cudaStream_t s);

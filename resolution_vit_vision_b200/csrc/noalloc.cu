@@ -93,13 +93,14 @@ extern "C" int vit_encode_noalloc(const void *patches, const int32_t *grid_thw, 
     const vit_weights_desc &d = h->desc;
 
     NA_TRY(vith::positions_launch_stack(grid_thw, n_images, P, d.patch_order, pos, merge_row, s));
-    CUtensorMap mPatch, mH, mF, mH4, mF4, mQKV;
+    CUtensorMap mPatch, mH, mF, mH4, mF4;
+    vith::AttnMaps mQKV;
     NA_TRY(vith::gemm_make_a_map(&mPatch, patches, P, VIT_PATCH_DIM));
     NA_TRY(vith::gemm_make_a_map(&mH, H, P, VIT_WIDTH));
     NA_TRY(vith::gemm_make_a_map(&mF, F, P, VIT_MLP));
     NA_TRY(vith::gemm_make_a_map(&mH4, H, M4, VIT_MERGE_DIM));
     NA_TRY(vith::gemm_make_a_map(&mF4, F, M4, VIT_MERGE_DIM));
-    NA_TRY(vith::attn_make_map(&mQKV, QKV, P));
+    NA_TRY(vith::attn_make_maps(&mQKV, QKV, P));
     CUtensorMap cX, cQKV, cF, cF4, cOut;
     NA_TRY(vith::gemm_make_c_map(&cX, X, P, VIT_WIDTH, VIT_EPI_ADD_F32));
     NA_TRY(vith::gemm_make_c_map(&cQKV, QKV, P, 3 * VIT_WIDTH, VIT_EPI_QKV_ROPE));
