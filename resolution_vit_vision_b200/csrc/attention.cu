@@ -24,7 +24,7 @@
 
 namespace vitk {
 
-constexpr int kAttnThreads = 320;                 // 10 warps
+constexpr int kAttnThreads = 352;                 // 11 warps
 constexpr int kBQ = 128, kBKV = 112, kD = 80;     // query tile, key tile, head dim
 constexpr int kQTilesPerCta = 2;                  // query tiles A and B share every K/V tile
 constexpr int kKVStages = 4;
@@ -59,10 +59,11 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// Warp roles: 0 TMA producer, 1 MMA issuer, 2..5 softmax of query tile A, 6..9 of tile B (one
-// query row per thread). Each tile has its own score and P buffers, so S_x(j+1) = Q_x K_(j+1)^T
-// runs on the tensor core while the softmax warpgroup is still turning S_x(j) into P_x(j).
-// 10 warps put 3 warps on two of the SM's four sub-partitions (16K registers each), which caps
+// Warp roles: 0 TMA producer; 1 and 2 issue the tensor-core products of query tile A and B
+// (one thread each, so neither tile's products wait behind the other's events); 3..6 softmax of
+// tile A, 7..10 of tile B (one query row per thread). Each tile has its own score and P buffers,
+// so S_x(j+1) = Q_x K_(j+1)^T runs while the softmax warpgroup still turns S_x(j) into P_x(j).
+// 11 warps put 3 warps on three of the SM's four sub-partitions (16K registers each), which caps
 // a thread at 168 registers.
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tkv,
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int s = 0; s < kKVStages; ++s) {
             mbar_init(k_full + s, 1);
             mbar_init(v_full + s, 1);
-            mbar_init(kv_empty + s, 1);
+            mbar_init(kv_empty + s, 2);              // released by both tiles' issuers
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(s_full + x, 1);
@@ -141,22 +142,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                 2 * VIT_WIDTH + head * kD + c * 16, r0);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 2) {
         if (lane == 0 && seg_len > 0) {
+            const int x = warp - 1;                                // query tile of this issuer
             constexpr uint32_t idS = idesc_bf16(kBQ, kBKV, false, false);
             constexpr uint32_t idO = idesc_bf16(kBQ, kD, false, true);   // V is N(=head dim)-major
-            const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
-            auto issue_s = [&](int x, int j) {    // S_x = Q_x K_j^T
+            const uint32_t qa = smem_u32(sQ) + x * kQBytes, ka = smem_u32(sK), va = smem_u32(sV);
+            auto issue_s = [&](int j) {          // S_x = Q_x K_j^T
                 const int st = j % kKVStages;
 #pragma unroll
                 for (int c = 0; c < 5; ++c) {
-                    const uint64_t da = smem_desc(qa + x * kQBytes + c * kQBox, 16, 256, kSwizzle32B);
+                    const uint64_t da = smem_desc(qa + c * kQBox, 16, 256, kSwizzle32B);
                     const uint64_t db = smem_desc(ka + st * kKVBytes + c * kKVBox, 16, 256, kSwizzle32B);
                     mma_bf16_ss(tmem + col_s(x), da, db, idS, c > 0 ? 1u : 0u);
                 }
                 mma_commit(s_full + x);
             };
-            auto issue_pv = [&](int x, int j) {   // O_x += P_x V_j, P_x read from TMEM (8 columns per 16 keys)
+            auto issue_pv = [&](int j) {         // O_x += P_x V_j, P_x read from TMEM (8 columns per 16 keys)
                 const int st = j % kKVStages;
 #pragma unroll
                 for (int kk = 0; kk < kBKV / 16; ++kk) {
@@ -164,37 +166,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     mma_bf16_ts(tmem + col_o(x), tmem + col_p(x) + kk * 8, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(o_done + x);
+                mma_commit(kv_empty + st);
             };
-            bool ok = mbar_wait(q_full, 0, wc) && mbar_wait(k_full, 0, wc);
+            auto wait_k = [&](int j) { return mbar_wait(k_full + j % kKVStages, (j / kKVStages) & 1, wc); };
+            bool ok = mbar_wait(q_full, 0, wc) && wait_k(0);
             if (ok) {
                 tc_fence_after();
-                issue_s(0, 0);
-                issue_s(1, 0);
+                issue_s(0);
             }
             for (int j = 0; ok && j < n_kv; ++j) {
-                const int st = j % kKVStages;
-                const uint32_t ph = j & 1;
-                if (j + 1 < n_kv) {
-                    // the next scores as soon as each softmax warpgroup has read this step's
-                    const int st1 = (j + 1) % kKVStages;
-                    if (!mbar_wait(k_full + st1, ((j + 1) / kKVStages) & 1, wc) || !mbar_wait(s_free, ph, wc)) break;
+                if (j + 1 < n_kv) {   // next scores once this tile's softmax has read S_x(j)
+                    if (!mbar_wait(s_free + x, j & 1, wc) || !wait_k(j + 1)) break;
                     tc_fence_after();
-                    issue_s(0, j + 1);
-                    if (!mbar_wait(s_free + 1, ph, wc)) break;
-                    tc_fence_after();
-                    issue_s(1, j + 1);
+                    issue_s(j + 1);
                 }
-                if (!mbar_wait(p_full, ph, wc) || !mbar_wait(v_full + st, (j / kKVStages) & 1, wc)) break;
+                if (!mbar_wait(p_full + x, j & 1, wc) ||
+                    !mbar_wait(v_full + j % kKVStages, (j / kKVStages) & 1, wc))
+                    break;
                 tc_fence_after();
-                issue_pv(0, j);
-                if (!mbar_wait(p_full + 1, ph, wc)) break;
-                tc_fence_after();
-                issue_pv(1, j);
-                mma_commit(kv_empty + st);
+                issue_pv(j);
             }
         }
     } else if (seg_len > 0) {
-        const int x = (warp - 2) >> 2;                             // query tile of this warpgroup
+        const int x = (warp - 3) >> 2;                             // query tile of this warpgroup
         const int quarter = warp & 3;                              // TMEM lanes 32*quarter ..
         const int r = quarter * 32 + lane;                         // query row inside the tile
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -204,8 +198,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
+        // Ping-pong: the two warpgroups take turns for the exponentials (named barriers 2 and 3),
+        // so one group's loads, max and stores run while the other keeps the MUFU busy.
+        // Group A goes first; B's initial arrive on barrier 2 opens A's first turn.
+        const int my_turn = 2 + x, their_turn = 3 - x;
+        if (x == 1) named_bar_arrive(2, 256);
         for (int j = 0; j < n_kv; ++j) {
-            if (!mbar_wait(s_full + x, j & 1, wc)) { ok = false; break; }
+            // a failed (timed-out) wait does not leave the loop: both groups must keep taking
+            // their turns on the named barriers; the results are then discarded
+            if (!mbar_wait(s_full + x, j & 1, wc)) ok = false;
             tc_fence_after();
             uint32_t sr[112];
             tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(sr));
@@ -235,47 +236,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float mx =
                 fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
                 scale_log2;
-            // P_x(j-1) V_(j-1) must be complete before O_x is rescaled or P_x is overwritten
-            if (j > 0) {
-                if (!mbar_wait(o_done + x, (j - 1) & 1, wc)) { ok = false; break; }
-                tc_fence_after();
-            }
+            // the rescale decision needs no tensor memory; O itself is scaled after the
+            // exponentials, once P_x(j-1) V_(j-1) has completed
             const bool need = mx > m_used + kRescaleThreshold;
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-                const float alpha = need ? ex2(m_used - mx) : 1.0f;
-                l *= alpha;
-#pragma unroll
-                for (int c = 0; c < 5; ++c) {
-                    uint32_t o[16];
-                    tmem_ld16(tO + c * 16, o);
-                    tmem_wait_ld();
-                    reg_fence16(o);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st16(tO + c * 16, o);
-                }
-                tmem_wait_st();
-            }
+            const float alpha = (j > 0 && need) ? ex2(m_used - mx) : 1.0f;
+            l *= alpha;
             if (need) m_used = mx;
             const float neg_m = -m_used;
             float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[56];
+            named_bar_sync(my_turn, 256);                           // this group's turn
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {   // keys [0, 64) and [64, 112) (+ 16 zero pad)
-                uint32_t pk[32];
-#pragma unroll
-                for (int k = 0; k < 64; k += 2) {
-                    const int kk = 64 * half + k;
-                    float p0 = 0.f, p1 = 0.f;
-                    if (kk < kBKV) {
-                        p0 = ex2(fmaf(__uint_as_float(sr[kk]), scale_log2, neg_m));
-                        p1 = ex2(fmaf(__uint_as_float(sr[kk + 1]), scale_log2, neg_m));
-                    }
-                    r8[(k >> 1) & 7] += p0 + p1;
-                    pk[k >> 1] = pack_bf16x2(p0, p1);
-                }
-                tmem_st32(tP + 32 * half, pk);
+            for (int k = 0; k < kBKV; k += 2) {
+                const float p0 = ex2(fmaf(__uint_as_float(sr[k]), scale_log2, neg_m));
+                const float p1 = ex2(fmaf(__uint_as_float(sr[k + 1]), scale_log2, neg_m));
+                r8[(k >> 1) & 7] += p0 + p1;
+                pk[k >> 1] = pack_bf16x2(p0, p1);
             }
+            // hand the MUFU to the other group (B's arrive after its last turn has no partner)
+            if (x == 0 || j + 1 < n_kv) named_bar_arrive(their_turn, 256);
             l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+            // P_x(j-1) V_(j-1) must be complete before O_x is rescaled or P_x is overwritten
+            if (j > 0) {
+                if (!mbar_wait(o_done + x, (j - 1) & 1, wc)) ok = false;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+                    for (int c = 0; c < 5; ++c) {
+                        uint32_t o[16];
+                        tmem_ld16(tO + c * 16, o);
+                        tmem_wait_ld();
+                        reg_fence16(o);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st16(tO + c * 16, o);
+                    }
+                }
+            }
+            tmem_st32(tP, pk);
+            tmem_st16(tP + 32, pk + 32);
+            {
+                uint32_t pad[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pad[e] = pk[48 + e];
+                tmem_st8(tP + 48, pad);
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(p_full + x);
