@@ -37,6 +37,9 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--shard", action="store_true",
+                    help="N > 1: split one batch across the ranks by image (strong scaling)")
+    ap.add_argument("--no-graph", action="store_true", help="launch every kernel instead of replaying a CUDA graph")
     ap.add_argument("--depth", type=int, default=None,
                     help="override the tower depth (profiling aid: small ncu captures of one layer)")
     return ap.parse_args()
@@ -230,10 +233,15 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
+    from resolution_vit_vision_b200 import dist as vd
+    import dataclasses
     wl = syn.WORKLOADS[args.workload]
     if args.depth is not None:
-        import dataclasses
         wl = dataclasses.replace(wl, depth=args.depth)
+    P_job = sum(t * h * w for t, h, w in wl.grids)          # patches of one whole batch
+    if args.shard and world > 1:                              # this rank's images of the one batch
+        _, my_grids, _ = vd.shard(wl.grids, rank, world, wl.depth)
+        wl = dataclasses.replace(wl, grids=tuple(my_grids))
     P, M4, flops_launch, ln_bytes, flops_total = work_model(wl.grids, wl.depth, wl.out_dim)
     wts = nv.random_weights_device(wl.depth, wl.out_dim, seed=wl.seed + 17 * rank, device=dev)
     g = torch.Generator(device=dev)
@@ -241,6 +249,8 @@ def main():
     patches = (torch.rand((P, syn.PATCH_K), generator=g, device=dev) * 2 - 1).to(torch.bfloat16)
     enc = nv.VisionEncoder(wts, wl.out_dim)
     enc.reserve(P)
+    if not args.no_graph:
+        enc.graph_enable(True)     # repeated encodes replay one recorded CUDA graph
     out = torch.empty((M4, wl.out_dim), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)   # > 126 MB L2
     stream = torch.cuda.current_stream()
@@ -282,10 +292,7 @@ def main():
     clocks = clk.stop() if clk else None
     # the same K steps again with an event pair around every kernel (per-kernel roofline)
     ms_prof, _, prof = timed_steps(True)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = vd.max_over_ranks(ms, device=dev)
     assert enc.device_status() == 0
 
     # ---- e2e: host (pinned) patches in, host tokens out, through vit_encode_host
@@ -301,11 +308,7 @@ def main():
         enc.encode_host(hp, wl.grids, ho)
         ev2[i][1].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in ev2]))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = vd.max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev2])), device=dev)
 
     pk, pk_kind = peaks()
     tc_peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
@@ -329,18 +332,22 @@ def main():
             "unit": "TFLOP/s", "frac": kernels[top]["frac"], "traffic": ncu_traffic(top),
             "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside the step)"}
 
+    strong = args.shard and world > 1
+    units = P_job if strong else world * P_job                # patches all ranks processed per step
     if rank == 0:
-        line = {"metric": METRIC, "value": world * P / (ms * 1e-3), "unit": "patches/s", "n_gpus": world,
+        line = {"metric": METRIC, "value": units / (ms * 1e-3), "unit": "patches/s", "n_gpus": world,
                 "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "scaling": "strong" if strong else "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded random weights N(0,0.02), patches U[-1,1])",
                 "config": {"workload": f"{wl.name}: {wl.description}", "patches": P, "merged": M4,
                            "depth": wl.depth, "out_dim": wl.out_dim, "l2": "flushed between steps (256 MB write)",
-                           "parallelism": f"dp{world} (images independent; weak scaling)"},
-                "merged_tokens_per_s": world * M4 / (ms * 1e-3),
+                           "parallelism": f"dp{world} (images independent; " +
+                                          ("one batch split by image)" if strong else "one batch per rank)"),
+                           "cuda_graph": not args.no_graph},
+                "merged_tokens_per_s": units / 4 / (ms * 1e-3),
                 "tc_peak_frac": achieved_total / tc_peak,
                 "tflops": achieved_total,
-                "e2e": {"value": world * P / (e2e_ms * 1e-3), "unit": "patches/s",
+                "e2e": {"value": units / (e2e_ms * 1e-3), "unit": "patches/s",
                         "h2d_bytes_per_step": P * syn.PATCH_K * 2, "d2h_bytes_per_step": M4 * wl.out_dim * 2,
                         "ms_per_step": e2e_ms},
                 "gpu_launches": int(launches),

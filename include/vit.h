@@ -127,6 +127,15 @@ int vit_reserve(vit_handle *h, int64_t max_patches);
 int vit_encode(const void *patches, const int32_t *grid_thw, int n_images, vit_handle *h,
                void *out, void *stream);
 
+/* CUDA-graph replay for repeated encodes (off by default). When enabled, the first vit_encode
+ * with a given (grid_thw values, patches pointer, out pointer) records its whole launch sequence
+ * into a CUDA graph on a private stream (nothing runs during the recording) and launches that
+ * graph on `stream`; later calls with the same signature replay it as one launch. Up to 4
+ * signatures are kept (least recently used evicted); growing the workspace or disabling drops
+ * them. The inputs are read when the graph runs, so new data in the same buffers is encoded.
+ * Profiling (vit_profile_enable) bypasses the graphs. */
+int vit_graph_enable(vit_handle *h, int enable);
+
 /* vit_encode with HOST patches and HOST out (pinned memory gives asynchronous copies): copies
  * the patches into the handle's workspace, encodes, copies the tokens back, all on `stream`.
  * The host buffers must stay valid until the stream reaches that point. */

@@ -64,6 +64,12 @@ int vit_op_layernorm(const float *X, const void *gamma, const void *beta, void *
 int vit_op_attention(const void *qkv, int64_t P, const int32_t *cu_seqlens, int n_seg, void *out,
                      int32_t *dev_status, void *stream);
 
+/* Bounded-wait self-test (the failure path of every tensor-core kernel's mbarrier waits, run on
+ * purpose and without any fault): one CTA waits on a barrier nothing arrives on; each wait gives
+ * up after limit_cycles SM cycles (1000 .. 4e9), the kernel writes VIT_ERR_TIMEOUT to *dev_status
+ * (device int32, required) and ends normally, leaving the context usable. */
+int vit_op_wait_selftest(int32_t *dev_status, int64_t limit_cycles, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

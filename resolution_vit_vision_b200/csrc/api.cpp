@@ -136,6 +136,8 @@ void prof_collect(vit_handle *h) {
     h->ev_used = 0;
 }
 
+void graph_clear(vit_handle *h);
+
 int ensure_workspace(vit_handle *h, int64_t P) {
     if (P <= h->ws_patches && h->ws) return VIT_OK;
     const int64_t Pn = P > 0 ? P : 1;
@@ -158,6 +160,7 @@ int ensure_workspace(vit_handle *h, int64_t P) {
     const size_t oSt = take(256);
     if (h->ws) {
         cudaDeviceSynchronize();
+        graph_clear(h);           // recorded graphs point into the old workspace
         cudaFree(h->ws);
         h->ws = nullptr;
     }
@@ -305,6 +308,78 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
     return VIT_OK;
 }
 
+void graph_clear(vit_handle *h) {
+    for (auto &g : h->graphs)
+        if (g.exec) cudaGraphExecDestroy(g.exec);
+    h->graphs.clear();
+}
+
+// vit_encode through a CUDA graph: the first call with a given (grid, patches, out) records the
+// whole launch sequence on a private stream and instantiates it; later calls replay it on the
+// caller's stream (one launch instead of ~229). At most kGraphCache signatures are kept.
+constexpr size_t kGraphCache = 4;
+
+int encode_graph(vit_handle *h, const void *patches, const int32_t *grid, int n_images, int64_t P, void *out,
+                 cudaStream_t s) {
+    std::vector<int32_t> key(grid, grid + 3 * n_images);
+    for (auto &g : h->graphs) {
+        if (g.patches == patches && g.out == out && g.grid == key) {
+            if (cudaGraphLaunch(g.exec, s) != cudaSuccess) return VIT_ERR_CUDA;
+            g.last_use = ++h->graph_clock;
+            h->launches += g.launches;
+            h->last_stream = s;
+            return VIT_OK;
+        }
+    }
+    if (!h->capture_stream &&
+        cudaStreamCreateWithFlags(&h->capture_stream, cudaStreamNonBlocking) != cudaSuccess)
+        return VIT_ERR_CUDA;
+    if (!h->rope_ready) {   // the once-per-workspace table is not part of the replayed graph
+        int rc = vith::rope_table_launch(h->rope_cs, VIT_MAX_SIDE, s);
+        if (rc != VIT_OK) return rc;
+        ++h->launches;
+        h->rope_ready = true;
+    }
+    // the caller's earlier work on `s` must precede the replay, which runs on `s` itself; the
+    // capture only records, so nothing else orders it
+    if (cudaStreamBeginCapture(h->capture_stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+        return VIT_ERR_CUDA;
+    const int64_t n0 = h->launches;
+    int rc = encode_device(h, patches, grid, n_images, P, out, h->capture_stream);
+    cudaGraph_t graph = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(h->capture_stream, &graph);
+    const int64_t recorded = h->launches - n0;
+    h->launches = n0;
+    if (rc != VIT_OK || e != cudaSuccess || !graph) {
+        if (graph) cudaGraphDestroy(graph);
+        cudaGetLastError();
+        return rc != VIT_OK ? rc : VIT_ERR_CUDA;
+    }
+    cudaGraphExec_t exec = nullptr;
+    const cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (ie != cudaSuccess) return VIT_ERR_CUDA;
+    if (h->graphs.size() == kGraphCache) {   // evict the least recently used signature
+        size_t lru = 0;
+        for (size_t i = 1; i < h->graphs.size(); ++i)
+            if (h->graphs[i].last_use < h->graphs[lru].last_use) lru = i;
+        cudaGraphExecDestroy(h->graphs[lru].exec);
+        h->graphs.erase(h->graphs.begin() + lru);
+    }
+    vit_handle::GraphEntry g;
+    g.grid = std::move(key);
+    g.patches = patches;
+    g.out = out;
+    g.exec = exec;
+    g.launches = recorded;
+    g.last_use = ++h->graph_clock;
+    h->graphs.push_back(std::move(g));
+    if (cudaGraphLaunch(exec, s) != cudaSuccess) return VIT_ERR_CUDA;
+    h->launches += recorded;
+    h->last_stream = s;
+    return VIT_OK;
+}
+
 }  // namespace
 
 // ============================================================================ C ABI
@@ -385,6 +460,8 @@ int vit_weights_create(const vit_weights_desc *d, vit_handle **out) {
 void vit_weights_destroy(vit_handle *h) {
     if (!h) return;
     cudaDeviceSynchronize();
+    graph_clear(h);
+    if (h->capture_stream) cudaStreamDestroy(h->capture_stream);
     for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
     if (h->ws) cudaFree(h->ws);
     delete h;
@@ -404,7 +481,16 @@ int vit_encode(const void *patches, const int32_t *grid_thw, int n_images, vit_h
     if (!aligned16(patches) || !aligned16(out)) return VIT_ERR_ALIGN;
     rc = ensure_workspace(h, P);
     if (rc != VIT_OK) return rc;
-    return encode_device(h, patches, grid_thw, n_images, P, out, static_cast<cudaStream_t>(stream));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!h->graph_on || h->prof) return encode_device(h, patches, grid_thw, n_images, P, out, s);
+    return encode_graph(h, patches, grid_thw, n_images, P, out, s);
+}
+
+int vit_graph_enable(vit_handle *h, int enable) {
+    if (!h) return VIT_ERR_ARG;
+    h->graph_on = enable != 0;
+    if (!h->graph_on) graph_clear(h);
+    return VIT_OK;
 }
 
 int vit_encode_host(const void *host_patches, const int32_t *grid_thw, int n_images, vit_handle *h, void *host_out,
@@ -533,6 +619,11 @@ int vit_op_attention(const void *qkv, int64_t P, const int32_t *cu_seqlens, int 
     const int rc = vith::attn_make_maps(&t, qkv, P);
     if (rc != VIT_OK) return rc;
     return vith::attn_launch(t, cu_seqlens, n_seg, out, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+int vit_op_wait_selftest(int32_t *dev_status, int64_t limit_cycles, void *stream) {
+    if (!dev_status || limit_cycles < 1000 || limit_cycles > 4000000000LL) return VIT_ERR_ARG;
+    return vith::wait_selftest_launch(dev_status, limit_cycles, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -48,4 +48,18 @@ struct vit_handle {
     double prof_ms[vith::kProfClasses] = {};
     int64_t prof_n[vith::kProfClasses] = {};
     cudaStream_t last_stream = nullptr;
+
+    // CUDA-graph replay of vit_encode (opt-in): the last few (grid, patches, out) signatures
+    struct GraphEntry {
+        std::vector<int32_t> grid;
+        const void *patches = nullptr;
+        void *out = nullptr;
+        cudaGraphExec_t exec = nullptr;
+        int64_t launches = 0;
+        uint64_t last_use = 0;
+    };
+    bool graph_on = false;
+    std::vector<GraphEntry> graphs;
+    uint64_t graph_clock = 0;
+    cudaStream_t capture_stream = nullptr;
 };

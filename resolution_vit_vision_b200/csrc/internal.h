@@ -47,6 +47,7 @@ int attn_launch_stack(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg
                       cudaStream_t s);
 int positions_launch_stack(const int32_t *grid_thw, int n_images, int64_t P, int patch_order, int32_t *pos,
                            int32_t *merge_row, cudaStream_t s);
+int wait_selftest_launch(int32_t *status, long long limit, cudaStream_t s);
 int mrope_launch(const int32_t *ids, int64_t L, const int32_t *grid_thw, int n_grids, int32_t *out, int32_t *delta,
                  int32_t *status, cudaStream_t s);
 

@@ -246,9 +246,34 @@ __global__ void __launch_bounds__(kMropeThreads)
     if (tid == 0 && delta) *delta = n_runs > 0 ? -s_shift[n_runs - 1] : 0;
 }
 
+// ------------------------------------------------------------------------------ wait self-test
+// Exercises the bounded-wait path on the GPU without any fault: every thread waits on an
+// mbarrier that nothing arrives on. Each wait must give up after `limit` cycles (or as soon as
+// another thread has raised the abort flag), write VIT_ERR_TIMEOUT to *status and return, so the
+// kernel ends normally and the context stays usable.
+__global__ void wait_selftest_kernel(int32_t *status, long long limit) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    WaitCtx wc{&abort_flag, status};
+    wc.limit = limit;
+    if (mbar_wait(&bar, 0, wc) && status) atomicExch(status, -1);   // a wait with no arrival succeeded
+}
+
 }  // namespace vitk
 
 namespace vith {
+
+int wait_selftest_launch(int32_t *status, long long limit, cudaStream_t s) {
+    vitk::wait_selftest_kernel<<<1, 64, 0, s>>>(status, limit);
+    return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
+}
+
 
 int layernorm_launch(const float *X, const void *gamma, const void *beta, void *Y, int64_t rows, float eps,
                      const int32_t *out_row, cudaStream_t s) {

@@ -76,6 +76,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
 struct WaitCtx {
     volatile int *abort;   // shared memory
     int32_t *status;       // global, may be null
+    long long limit = kWaitCycles;
 };
 
 static __device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, WaitCtx c) {
@@ -84,7 +85,7 @@ static __device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, Wa
     while (!mbar_try_wait_sleep(bar, parity)) {
         if ((++n & 3u) == 0) {
             if (*c.abort) return false;
-            if (clock64() - t0 > kWaitCycles) {
+            if (clock64() - t0 > c.limit) {
                 *c.abort = 1;
                 if (c.status) atomicExch(c.status, VIT_ERR_TIMEOUT);
                 return false;

@@ -49,6 +49,7 @@ _SIGS = {
     "mrope_index": (c_int, [c_void_p, c_int64, c_i32p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "vit_device_status": (c_int, [c_void_p, c_void_p, c_i32p]),
     "vit_launch_count": (c_int64, [c_void_p]),
+    "vit_graph_enable": (c_int, [c_void_p, c_int]),
     "vit_profile_enable": (c_int, [c_void_p, c_int]),
     "vit_profile_read": (c_int, [c_void_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_int64), c_int]),
     "vit_profile_name": (ctypes.c_char_p, [c_int]),
@@ -58,6 +59,7 @@ _SIGS = {
     "vit_op_positions": (c_int, [c_i32p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "vit_op_layernorm": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_float, c_void_p, c_void_p]),
     "vit_op_attention": (c_int, [c_void_p, c_int64, c_i32p, c_int, c_void_p, c_void_p, c_void_p]),
+    "vit_op_wait_selftest": (c_int, [c_void_p, c_int64, c_void_p]),
 }
 
 _lib = None
@@ -217,6 +219,9 @@ class VisionEncoder:
         check(lib().vit_device_status(self._h, _stream(stream), ctypes.byref(v)), "vit_device_status")
         return v.value
 
+    def graph_enable(self, on: bool = True):
+        check(lib().vit_graph_enable(self._h, 1 if on else 0), "vit_graph_enable")
+
     def launch_count(self) -> int:
         return int(lib().vit_launch_count(self._h))
 
@@ -282,3 +287,7 @@ def op_attention(qkv, cu_seqlens: Sequence[int], out, status=None, stream=None):
     check(lib().vit_op_attention(_ptr(qkv), qkv.shape[0], cu.ctypes.data_as(c_i32p), cu.shape[0] - 1, _ptr(out),
                                  _ptr(status), _stream(stream)), "vit_op_attention")
     return out
+
+
+def op_wait_selftest(status, limit_cycles: int, stream=None):
+    check(lib().vit_op_wait_selftest(_ptr(status), int(limit_cycles), _stream(stream)), "vit_op_wait_selftest")

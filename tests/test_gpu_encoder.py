@@ -155,3 +155,45 @@ def test_video_batch_sampled():
     one = [(1, 32, 32)]
     g1, *_ = _run(one, wl.depth, wl.out_dim, wl.seed, patches=patches[3072:4096], wts=wts)
     np.testing.assert_array_equal(g1, got[768:1024])
+
+
+def test_graph_replay_matches_direct_launches():
+    grids = [(1, 8, 12), (2, 4, 6)]
+    wts = syn.make_weights(2, 1536, 14)
+    enc = nv.VisionEncoder(nv.weights_to_device(wts), 1536)
+    p1 = bf16_bits_to_torch(syn.make_patches(grids, 14))
+    ref = to_np(enc.encode(p1, grids))
+    enc.graph_enable(True)
+    out = torch.empty((ref.shape[0], 1536), dtype=torch.bfloat16, device=DEV)
+    n0 = enc.launch_count()
+    enc.encode(p1, grids, out=out)                 # records and launches
+    enc.encode(p1, grids, out=out)                 # replays
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_np(out), ref)
+    assert (enc.launch_count() - n0) % 2 == 0 and enc.launch_count() > n0
+    # new data in the same buffers is encoded by the replay
+    p2 = bf16_bits_to_torch(syn.make_patches(grids, 15))
+    p1.copy_(p2)
+    enc.encode(p1, grids, out=out)
+    enc.graph_enable(False)
+    ref2 = to_np(enc.encode(p2, grids))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_np(out), ref2)
+    assert enc.device_status() == 0
+
+
+@pytest.mark.slow
+def test_hires_1792_single_segment():
+    # 16384 patches in one attention segment: the whole image through the oracle at depth 1
+    # (the oracle's cost at depth 32 is out of reach), and the full-depth run in the benchmark's
+    # configuration must stay finite with the printed shape
+    wl = syn.WORKLOADS["hires_1792"]
+    wts1 = syn.make_weights(1, wl.out_dim, wl.seed)
+    got, _, patches, _ = _run(wl.grids, 1, wl.out_dim, wl.seed, wts=wts1)
+    ref = vo.vit_encode(patches, wl.grids, wts1)
+    assert_encoder_close(got, ref, "1792^2 depth 1")
+    full = nv.VisionEncoder(nv.random_weights_device(wl.depth, wl.out_dim, wl.seed), wl.out_dim)
+    out = full.encode(bf16_bits_to_torch(patches), wl.grids)
+    assert full.device_status() == 0
+    o = to_np(out)
+    assert o.shape == (4096, 3584) and np.isfinite(o).all()

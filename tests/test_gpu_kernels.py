@@ -219,3 +219,16 @@ def test_mrope_empty_prompt():
     out, delta = nv.mrope_index(t, None)
     torch.cuda.synchronize()
     assert out.shape == (3, 0) and int(delta.item()) == 0
+
+
+# ------------------------------------------------------------------ bounded waits
+def test_bounded_wait_times_out_and_context_survives():
+    # a wait that nothing satisfies must end with VIT_ERR_TIMEOUT, not hang; the GPU stays usable
+    st = _status()
+    nv.op_wait_selftest(st, 2_000_000)
+    torch.cuda.synchronize()
+    assert int(st.item()) == nv.VIT_ERR_TIMEOUT
+    a, b = _bits((130, 64), 61, 1.0), _bits((256, 64), 62, 0.02)
+    C = torch.empty((130, 256), device=DEV)
+    nv.op_gemm(bf16_bits_to_torch(a), bf16_bits_to_torch(b), None, C, nv.EPI_STORE_F32)
+    assert_fp32_close(to_np(C), vo.linear(a, b), 1e-4, "gemm after timeout test")
