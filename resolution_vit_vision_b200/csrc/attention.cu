@@ -226,17 +226,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int k = 0; k < kBKV; ++k)
                     if (k >= kv_valid) sr[k] = __float_as_uint(-INFINITY);
             }
-            // row max: eight independent three-input max chains
             float m8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) m8[i] = __uint_as_float(sr[i]);
 #pragma unroll
-            for (int k = 8; k + 16 <= kBKV; k += 16)
+            for (int k = 8; k < kBKV; k += 8)
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    m8[i] = fmax3(m8[i], __uint_as_float(sr[k + i]), __uint_as_float(sr[k + 8 + i]));
-#pragma unroll
-            for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], __uint_as_float(sr[kBKV - 8 + i]));
+                for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], __uint_as_float(sr[k + i]));
             const float mx =
                 fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
                 scale_log2;
@@ -247,16 +243,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             l *= alpha;
             if (need) m_used = mx;
             const float neg_m = -m_used;
-            uint32_t pk[56];
             float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[56];
             named_bar_sync(my_turn, 256);                           // this group's turn
 #pragma unroll
-            for (int k = 0; k < kBKV; k += 2) {   // per pair: x = s * scale - m, 2^x, sum, bf16 pack
-                float x0, x1;
-                ffma2(x0, x1, __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]), scale_log2, scale_log2, neg_m,
-                      neg_m);
-                const float p0 = ex2(x0), p1 = ex2(x1);
-                fadd2(r8[(k >> 1) & 3], r8[4 + ((k >> 1) & 3)], p0, p1);
+            for (int k = 0; k < kBKV; k += 2) {
+                const float p0 = ex2(fmaf(__uint_as_float(sr[k]), scale_log2, neg_m));
+                const float p1 = ex2(fmaf(__uint_as_float(sr[k + 1]), scale_log2, neg_m));
+                r8[(k >> 1) & 7] += p0 + p1;
                 pk[k >> 1] = pack_bf16x2(p0, p1);
             }
             // hand the MUFU to the other group (B's arrive after its last turn has no partner)
