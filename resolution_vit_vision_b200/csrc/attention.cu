@@ -246,12 +246,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             uint32_t pk[56];
             named_bar_sync(my_turn, 256);                           // this group's turn
+            // groups of four pairs: eight independent exponentials in flight before their results
+            // are summed and packed, so the MUFU latency overlaps within one thread
 #pragma unroll
-            for (int k = 0; k < kBKV; k += 2) {
-                const float p0 = ex2(fmaf(__uint_as_float(sr[k]), scale_log2, neg_m));
-                const float p1 = ex2(fmaf(__uint_as_float(sr[k + 1]), scale_log2, neg_m));
-                r8[(k >> 1) & 7] += p0 + p1;
-                pk[k >> 1] = pack_bf16x2(p0, p1);
+            for (int k = 0; k < kBKV; k += 8) {
+                float p[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) p[e] = fmaf(__uint_as_float(sr[k + e]), scale_log2, neg_m);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) p[e] = ex2(p[e]);
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    r8[(e >> 1) + 4 * ((k >> 3) & 1)] += p[e] + p[e + 1];
+                    pk[(k + e) >> 1] = pack_bf16x2(p[e], p[e + 1]);
+                }
             }
             // hand the MUFU to the other group (B's arrive after its last turn has no partner)
             if (x == 0 || j + 1 < n_kv) named_bar_arrive(their_turn, 256);

@@ -287,6 +287,18 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
+// ---------------------------------------------------------------- register reallocation
+// Per-warpgroup register budget changes (all four warps of a warpgroup execute them). The
+// block's total never changes: what one warpgroup releases, another may take.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
