@@ -30,6 +30,19 @@ Readings of points the pages leave open (each is listed in the design doc):
 * patch_order 0 = 2x2-block order (per frame: bh, bw, dh, dw), 1 = raster order (h, w);
   the merged token concatenates its four patches in (dh, dw) = 00, 01, 10, 11 order;
 * merger LayerNorm eps 1e-6 (the same as the tower's), GELU exact.
+
+Windowed attention (the Qwen2.5-VL tower): "Qwen2.5-VL-7B-Instruct" (inference-research model
+record), architecture note: the same 32-block, 1280-wide tower as Qwen2-VL, but its blocks attend
+inside windows of 112 px, except four full-attention blocks at depths 7, 15, 23 and 31. Readings:
+
+* a window is 112 / 14 = 8 x 8 patches, tiled from the frame's top-left corner; windows on the
+  bottom and right borders are cut short (no padding tokens take part in the softmax);
+* window membership of a patch is (frame, h // 8, w // 8); each frame of a video is windowed on
+  its own; the window side is even, so a window never splits a 2x2 merge group;
+* the depths are 0-based block indices; the full-attention blocks attend per (image, frame) as
+  the Qwen2-VL tower does;
+* nothing else in the block changes (the page names no other difference), and the merged tokens
+  come out in the same order as without windows.
 """
 from __future__ import annotations
 
@@ -170,6 +183,25 @@ def patch_positions(grids, patch_order: int) -> Tuple[np.ndarray, np.ndarray]:
     return np.concatenate(hs), np.concatenate(ws)
 
 
+def window_groups(grids, patch_order: int, window: int) -> List[np.ndarray]:
+    """Row indices of every attention window: per image, per frame, the windows of window x window
+    patches tiled from the frame's top-left corner (border windows cut short) in raster order of
+    the windows; inside a window the rows keep their packed order. A patch at (h, w) belongs to
+    window (h // window, w // window) of its frame."""
+    if window < 2 or window % 2:
+        raise ValueError("window side must be even and >= 2 (whole 2x2 merge groups)")
+    out, row = [], 0
+    for t, h, w in check_grid(grids):
+        hp, wp = frame_positions(h, w, patch_order)
+        nwh, nww = -(-h // window), -(-w // window)
+        key = (hp // window) * nww + (wp // window)
+        for _ in range(t):
+            for k in range(nwh * nww):
+                out.append(row + np.nonzero(key == k)[0])
+            row += h * w
+    return out
+
+
 def merge_groups(grids, patch_order: int) -> np.ndarray:
     """Row indices [P/4, 4]: the four patches of each merged token, (dh, dw) = 00, 01, 10, 11,
     merged tokens per image, per frame, in (bh, bw) raster order."""
@@ -214,11 +246,23 @@ def varlen_attention(q, k, v, segs) -> np.ndarray:
     return out.reshape(P, WIDTH)
 
 
-def vit_block(x: np.ndarray, L: Dict, segs, hpos, wpos, eps: float) -> np.ndarray:
-    """Pre-norm block: x += proj(attn(rope(qkv(LN1 x)))) ; x += fc2(GELU(fc1(LN2 x)))."""
+def grouped_attention(q, k, v, groups) -> np.ndarray:
+    """Attention inside each group of rows (index arrays; every row in exactly one group): the
+    rows of a group attend to each other and to nothing else. Returns [P, 1280]."""
+    P = q.shape[0]
+    out = np.zeros((P, HEADS, HEAD_DIM), np.float64)
+    for idx in groups:
+        for i in range(HEADS):
+            out[idx, i] = attention(q[idx, i], k[idx, i], v[idx, i])
+    return out.reshape(P, WIDTH)
+
+
+def vit_block(x: np.ndarray, L: Dict, segs, hpos, wpos, eps: float, groups=None) -> np.ndarray:
+    """Pre-norm block: x += proj(attn(rope(qkv(LN1 x)))) ; x += fc2(GELU(fc1(LN2 x))).
+    Attention per segment, or inside each of ``groups`` (windows) when given."""
     h = layer_norm(x, L["ln1_w"], L["ln1_b"], eps)
     q, k, v = qkv_rope(h, L, hpos, wpos)
-    a = varlen_attention(q, k, v, segs)
+    a = varlen_attention(q, k, v, segs) if groups is None else grouped_attention(q, k, v, groups)
     x = x + linear(a, L["proj_w"], L["proj_b"])
     h = layer_norm(x, L["ln2_w"], L["ln2_b"], eps)
     x = x + linear(gelu_erf(linear(h, L["fc1_w"], L["fc1_b"])), L["fc2_w"], L["fc2_b"])
@@ -235,15 +279,19 @@ def merger(x: np.ndarray, grids, weights: Dict, eps: float, patch_order: int) ->
 
 
 def vit_encode(patches, grids, weights: Dict, depth: int = None, eps: float = 1e-6,
-               patch_order: int = 0, return_hidden: bool = False):
-    """Patches [P, 1176] + grid_thw -> merged tokens [P/4, out_dim] (float64)."""
+               patch_order: int = 0, return_hidden: bool = False, window: int = 0,
+               full_blocks: Sequence[int] = ()):
+    """Patches [P, 1176] + grid_thw -> merged tokens [P/4, out_dim] (float64).
+    window > 0: blocks whose index is not in full_blocks attend inside window x window patches."""
     g = check_grid(grids)
     segs = segments(g)
     hpos, wpos = patch_positions(g, patch_order)
+    groups = window_groups(g, patch_order, window) if window else None
     depth = len(weights["layers"]) if depth is None else depth
     x = patch_embed(patches, weights["pe_w"], weights.get("pe_b"))
     for l in range(depth):
-        x = vit_block(x, weights["layers"][l], segs, hpos, wpos, eps)
+        windowed = groups is not None and l not in full_blocks
+        x = vit_block(x, weights["layers"][l], segs, hpos, wpos, eps, groups if windowed else None)
     out = merger(x, g, weights, eps, patch_order)
     return (out, x) if return_hidden else out
 
