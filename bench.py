@@ -42,6 +42,10 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch every kernel instead of replaying a CUDA graph")
     ap.add_argument("--depth", type=int, default=None,
                     help="override the tower depth (profiling aid: small ncu captures of one layer)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="the windowed (Qwen2.5-VL) tower: window side in patches (8 = 112 px); 0 = Qwen2-VL")
+    ap.add_argument("--full-blocks", default="7,15,23,31",
+                    help="with --window: the full-attention blocks (0-based, comma-separated)")
     return ap.parse_args()
 
 
@@ -71,11 +75,23 @@ def segments_of(grids):
     return [h * w for t, h, w in grids for _ in range(t)]
 
 
-def work_model(grids, depth, out_dim):
+def windows_of(grids, window):
+    """Patches per attention window: window x window patches tiled from each frame's top-left
+    corner, border windows cut short."""
+    out = []
+    for t, h, w in grids:
+        rows = [min(window, h - a) for a in range(0, h, window)]
+        cols = [min(window, w - b) for b in range(0, w, window)]
+        out += [r * c for _ in range(t) for r in rows for c in cols]
+    return out
+
+
+def work_model(grids, depth, out_dim, window=0, full_blocks=()):
     """Algorithmic FLOPs (2 per multiply-add) and bytes per kernel launch class, per encode."""
     P = sum(t * h * w for t, h, w in grids)
     M4 = P // 4
     s2 = sum(n * n for n in segments_of(grids))
+    n_full = depth if not window else sum(1 for l in range(depth) if l in full_blocks)
     per_launch = {
         "patch_embed": 2.0 * P * 1176 * 1280,
         "qkv_rope": 2.0 * P * 1280 * 3840,
@@ -86,10 +102,12 @@ def work_model(grids, depth, out_dim):
         "merger_fc1": 2.0 * M4 * 5120 * 5120,
         "merger_fc2": 2.0 * M4 * 5120 * out_dim,
     }
+    if window:
+        per_launch["attention_window"] = 4.0 * 1280 * sum(n * n for n in windows_of(grids, window))
     ln_bytes = P * 1280 * (4 + 2) + 2 * 1280 * 2      # read fp32 row, write bf16 row, gamma/beta
     total = per_launch["patch_embed"] + per_launch["merger_fc1"] + per_launch["merger_fc2"] + depth * (
-        per_launch["qkv_rope"] + per_launch["attention"] + per_launch["out_proj"] + per_launch["fc1_gelu"] +
-        per_launch["fc2"])
+        per_launch["qkv_rope"] + per_launch["out_proj"] + per_launch["fc1_gelu"] + per_launch["fc2"]) + \
+        n_full * per_launch["attention"] + (depth - n_full) * per_launch.get("attention_window", 0.0)
     return P, M4, per_launch, ln_bytes, total
 
 
@@ -152,7 +170,7 @@ def _oracle_weights(depth, out_dim, seed):
     return _WCACHE[key]
 
 
-def cpu_baseline(wl, budget_s=25.0):
+def cpu_baseline(wl, budget_s=25.0, window=0, full_blocks=()):
     """The CPU oracle, as it stands, on a bounded sample of the workload: the smallest image of
     the batch through the full-depth tower (every image is independent, so this is a slice of the
     same job). Returns patches/s over the sample."""
@@ -172,7 +190,7 @@ def cpu_baseline(wl, budget_s=25.0):
     done = 0
     # a bounded number of passes: at least one, more while under the budget
     while True:
-        vo.vit_encode(patches, g, wts)
+        vo.vit_encode(patches, g, wts, window=window, full_blocks=full_blocks)
         done += 1
         el = time.perf_counter() - t0
         if el * (done + 1) / done > budget_s:
@@ -180,7 +198,8 @@ def cpu_baseline(wl, budget_s=25.0):
     el = time.perf_counter() - t0
     return {"value": done * P / el, "unit": "patches/s", "cores": int(cores), "kind": "oracle",
             "sample": f"image {i} of the batch (grid {tuple(g[0])}, {P} patches) through the full "
-                      f"depth-{wl.depth} fp64 oracle, {done} pass(es), {el:.1f} s"}
+                      f"depth-{wl.depth} fp64 oracle{' (windowed)' if window else ''}, {done} pass(es), "
+                      f"{el:.1f} s"}
 
 
 # ------------------------------------------------------------------------------ reference arm
@@ -190,13 +209,14 @@ def run_reference(args):
         return 0
     from resolution_vit_vision_b200 import synthetic as syn
     wl = syn.WORKLOADS[args.workload]
-    P, M4, _, _, _ = work_model(wl.grids, wl.depth, wl.out_dim)
+    full_blocks = tuple(int(x) for x in args.full_blocks.split(",") if x) if args.window else ()
+    P, M4, _, _, _ = work_model(wl.grids, wl.depth, wl.out_dim, args.window, full_blocks)
     # each step: one bounded sample (the smallest image of the batch through the full-depth
     # oracle); the run stops early once about three minutes of CPU time are spent
     vals = []
     t0 = time.perf_counter()
     for _ in range(max(1, args.steps)):
-        vals.append(cpu_baseline(wl, budget_s=0.0))
+        vals.append(cpu_baseline(wl, budget_s=0.0, window=args.window, full_blocks=full_blocks))
         if time.perf_counter() - t0 > 180.0:
             break
     v = statistics.median(x["value"] for x in vals)
@@ -204,7 +224,8 @@ def run_reference(args):
             "steps": len(vals), "warmup": 0, "ms_per_step": 1000.0 * P / v, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{wl.name}: {wl.description}", "patches": P, "merged": M4,
-                       "depth": wl.depth, "out_dim": wl.out_dim},
+                       "depth": wl.depth, "out_dim": wl.out_dim, "window": args.window,
+                       "full_blocks": list(full_blocks)},
             "merged_tokens_per_s": v / 4,
             "cpu_baseline": {"value": v, "unit": "patches/s", "cores": vals[0]["cores"], "kind": "oracle",
                              "sample": vals[0]["sample"]},
@@ -242,12 +263,14 @@ def main():
     if args.shard and world > 1:                              # this rank's images of the one batch
         _, my_grids, _ = vd.shard(wl.grids, rank, world, wl.depth)
         wl = dataclasses.replace(wl, grids=tuple(my_grids))
-    P, M4, flops_launch, ln_bytes, flops_total = work_model(wl.grids, wl.depth, wl.out_dim)
+    full_blocks = tuple(int(x) for x in args.full_blocks.split(",") if x) if args.window else ()
+    P, M4, flops_launch, ln_bytes, flops_total = work_model(wl.grids, wl.depth, wl.out_dim, args.window,
+                                                            full_blocks)
     wts = nv.random_weights_device(wl.depth, wl.out_dim, seed=wl.seed + 17 * rank, device=dev)
     g = torch.Generator(device=dev)
     g.manual_seed(wl.seed + 1000 + rank)
     patches = (torch.rand((P, syn.PATCH_K), generator=g, device=dev) * 2 - 1).to(torch.bfloat16)
-    enc = nv.VisionEncoder(wts, wl.out_dim)
+    enc = nv.VisionEncoder(wts, wl.out_dim, window=args.window, full_blocks=full_blocks)
     enc.reserve(P)
     if not args.no_graph:
         enc.graph_enable(True)     # repeated encodes replay one recorded CUDA graph
@@ -320,14 +343,25 @@ def main():
         avg = rec["ms"] / rec["launches"]
         k = {"ms_per_step": rec["ms"] / args.steps, "launches_per_step": rec["launches"] / args.steps,
              "avg_launch_ms": avg}
-        if name in flops_launch:
+        if name == "attention_window":   # HBM-bound: q, k, v read once, the output written once
+            k["tflops"] = flops_launch[name] / (avg * 1e-3) / 1e12
+            k["gbs"] = P * (3840 + 1280) * 2 / (avg * 1e-3) / 1e9
+            k["frac"] = k["gbs"] / pk["hbm_gbs"]
+        elif name in flops_launch:
             k["tflops"] = flops_launch[name] / (avg * 1e-3) / 1e12
             k["frac"] = k["tflops"] / tc_peak
         elif name == "layernorm":
             k["gbs"] = ln_bytes / (avg * 1e-3) / 1e9
             k["frac"] = k["gbs"] / pk["hbm_gbs"]
         kernels[name] = k
-    top = max((n for n in kernels if n in flops_launch), key=lambda n: kernels[n]["ms_per_step"])
+    if "attention" in kernels:   # exponentials: 16 heads x sum S^2 per launch, against 16 ex2 / clock / SM
+        sm_hz = 1e6 * (clocks["sm_mhz"] if clocks else 1965.0)   # sampled median, else the B200's max clock
+        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+        a = kernels["attention"]
+        a["exp_per_s"] = 16.0 * sum(n * n for n in segments_of(wl.grids)) / (a["avg_launch_ms"] * 1e-3)
+        a["mufu_frac"] = a["exp_per_s"] / (16.0 * n_sm * sm_hz)
+    top = max((n for n in kernels if n in flops_launch and n != "attention_window"),
+              key=lambda n: kernels[n]["ms_per_step"])
     roof = {"kernel": top, "bound": "tensor", "achieved": kernels[top]["tflops"], "peak": tc_peak,
             "unit": "TFLOP/s", "frac": kernels[top]["frac"], "traffic": ncu_traffic(top),
             "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside the step)"}
@@ -343,7 +377,8 @@ def main():
                            "depth": wl.depth, "out_dim": wl.out_dim, "l2": "flushed between steps (256 MB write)",
                            "parallelism": f"dp{world} (images independent; " +
                                           ("one batch split by image)" if strong else "one batch per rank)"),
-                           "cuda_graph": not args.no_graph},
+                           "cuda_graph": not args.no_graph,
+                           **({"window": args.window, "full_blocks": list(full_blocks)} if args.window else {})},
                 "merged_tokens_per_s": units / 4 / (ms * 1e-3),
                 "tc_peak_frac": achieved_total / tc_peak,
                 "tflops": achieved_total,
@@ -356,7 +391,7 @@ def main():
                 "kernels": kernels,
                 "clocks": clocks}
         if not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl)
+            line["cpu_baseline"] = cpu_baseline(wl, window=args.window, full_blocks=full_blocks)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

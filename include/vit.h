@@ -94,6 +94,17 @@ typedef struct {
     const void *lnq_w, *lnq_b; /* merger LayerNorm [1280]                                       */
     const void *m0_w, *m0_b;   /* merger Linear 1 [5120, 5120], [5120]                          */
     const void *m2_w, *m2_b;   /* merger Linear 2 [out_dim, 5120], [out_dim]                    */
+    /* Windowed attention, the Qwen2.5-VL tower ("Qwen2.5-VL-7B-Instruct", inference-research
+     * model record, architecture note: 112-px windows, full attention only at depths 7, 15, 23,
+     * 31). 0 (or zero-initialised): every block attends over its whole (image, frame) segment, the
+     * Qwen2-VL tower. window > 0: the side of a window in patches, even, 2..VIT_MAX_SIDE (8 =
+     * 112 px); windows tile each frame from its top-left corner, border windows are cut short,
+     * and a patch at (h, w) attends only to the patches of its window (h / window, w / window).
+     * Windows of up to 8 x 8 patches run on a dedicated kernel; larger ones on the segment kernel. */
+    int window;
+    const uint8_t *full_attention; /* HOST [depth] or NULL; copied by vit_weights_create. With
+                                      window > 0, block l attends over the whole frame where
+                                      full_attention[l] != 0 (Qwen2.5-VL: l = 7, 15, 23, 31) */
 } vit_weights_desc;
 
 typedef struct vit_handle vit_handle;  /* validated weight view + workspace + device status word */
@@ -122,8 +133,9 @@ int vit_reserve(vit_handle *h, int64_t max_patches);
  * frames in temporal order, each frame's patches in desc.patch_order. grid_thw: HOST int32
  * [n_images, 3] = (t, h, w) in patch units (h, w even). out: bf16 [P/4, out_dim]; row order =
  * images in grid_thw order, then t, then the merged (h/2, w/2) grid in raster order.
- * Attention is full within each (image, frame) segment and never crosses segments.
- * May allocate (synchronously) if the workspace is too small, see vit_reserve. */
+ * Attention is full within each (image, frame) segment and never crosses segments (inside
+ * windows for the windowed blocks of a handle made with desc.window > 0; the output order is the
+ * same). May allocate (synchronously) if the workspace is too small, see vit_reserve. */
 int vit_encode(const void *patches, const int32_t *grid_thw, int n_images, vit_handle *h,
                void *out, void *stream);
 
@@ -173,7 +185,8 @@ int mrope_index(const int32_t *input_ids, int64_t L, const int32_t *grid_thw, in
  *     it. Calls whose work overlaps on the GPU race with each other: issue them on one stream or
  *     order them. Nothing in the array needs clearing between calls: each buffer is fully
  *     written before it is read.
- *   - Arguments as for vit_encode; weights from vit_weights_create on the current device.
+ *   - Arguments as for vit_encode; weights from vit_weights_create on the current device, made
+ *     without windows (desc.window == 0; a windowed handle returns VIT_ERR_ARG).
  *     dev_status: int32 [1] device or NULL; a kernel wait that timed out writes VIT_ERR_TIMEOUT
  *     there (it is not cleared by the call). */
 #define VIT_NOALLOC_MAX_PATCHES 1024

@@ -64,6 +64,28 @@ int vit_op_layernorm(const float *X, const void *gamma, const void *beta, void *
 int vit_op_attention(const void *qkv, int64_t P, const int32_t *cu_seqlens, int n_seg, void *out,
                      int32_t *dev_status, void *stream);
 
+/* Window order of the windowed (Qwen2.5-VL) tower ("Qwen2.5-VL-7B-Instruct", inference-research
+ * model record, architecture note: 112-px windows). Rows in window order run, per image and frame,
+ * over the windows of window x window patches (window even, >= 2) in raster order, inside a window
+ * over its 2x2 merge groups in raster order, inside a group (dh, dw). For each window-order row r:
+ * pos[r] = (h << 16) | w inside its frame, src_row[r] = the row holding that patch when the images
+ * are packed in patch_order (0 block, 1 raster), merge_row[r] = its row in 2x2-block order. All
+ * three are int32 [P] device buffers (required). grid_thw: HOST [n_images, 3]. */
+int vit_op_window_positions(const int32_t *grid_thw, int n_images, int patch_order, int window, int32_t *pos,
+                            int32_t *merge_row, int32_t *src_row, void *stream);
+
+/* dst[r, :] = src[src_row[r], :] for rows of row_bytes bytes (a multiple of 16; src, dst
+ * 16-byte aligned). src_row: int32 [rows] device, each in range of src (not checked). */
+int vit_op_gather_rows(const void *src, const int32_t *src_row, void *dst, int64_t rows, int row_bytes,
+                       void *stream);
+
+/* Attention inside windows (same architecture note): qkv bf16 [P, 3840] with its rows in window
+ * order for the images of grid_thw (HOST [n_images, 3]); every window of window x window patches
+ * (window even, 2..8) is one segment, attended exactly as by vit_op_attention. out: bf16 [P, 1280]
+ * in the same row order. dev_status as for vit_op_attention. */
+int vit_op_window_attention(const void *qkv, const int32_t *grid_thw, int n_images, int window, void *out,
+                            int32_t *dev_status, void *stream);
+
 /* Bounded-wait self-test (the failure path of every tensor-core kernel's mbarrier waits, run on
  * purpose and without any fault): one CTA waits on a barrier nothing arrives on; each wait gives
  * up after limit_cycles SM cycles (1000 .. 4e9), the kernel writes VIT_ERR_TIMEOUT to *dev_status

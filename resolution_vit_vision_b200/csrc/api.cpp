@@ -72,9 +72,10 @@ int check_device() {
 // ============================================================================ handle
 namespace {
 
-const char *kProfNames[vith::kProfClasses] = {"patch_embed", "layernorm", "qkv_rope", "attention", "out_proj",
-                                        "fc1_gelu",    "fc2",       "merger_fc1", "merger_fc2", "positions"};
-enum ProfClass { P_PE, P_LN, P_QKV, P_ATT, P_PROJ, P_FC1, P_FC2, P_M0, P_M2, P_POS };
+const char *kProfNames[vith::kProfClasses] = {"patch_embed", "layernorm",  "qkv_rope",   "attention",
+                                              "out_proj",    "fc1_gelu",   "fc2",        "merger_fc1",
+                                              "merger_fc2",  "positions",  "attention_window"};
+enum ProfClass { P_PE, P_LN, P_QKV, P_ATT, P_PROJ, P_FC1, P_FC2, P_M0, P_M2, P_POS, P_WATT };
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -210,6 +211,11 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
     const int n_seg = static_cast<int>(cu.size()) - 1;
     if (n_seg > VIT_MAX_SEGMENTS) return VIT_ERR_LIMIT;
     const int64_t M4 = P / 4;
+    // windowed blocks: rows live in window order (window.cu); windows of up to 8 x 8 patches go to
+    // the packed window kernel, larger ones to the segment kernel with one segment per window
+    const int window = d.window;
+    std::vector<int32_t> cu_win;
+    if (window > 8) VIT_TRY(vith::window_cu_seqlens(grid, n_images, window, cu_win));
 
     if (!h->rope_ready) {
         ProfScope ps(h, s, P_POS);
@@ -217,15 +223,27 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
         ++nl;
         h->rope_ready = true;
     }
-    {
+    if (window == 0) {
         ProfScope ps(h, s, P_POS);
         VIT_TRY(vith::positions_launch(grid, n_images, P, d.patch_order, h->pos, h->merge_row, s));
         ++nl;
+    } else {
+        // the gather's source rows sit in the QKV buffer and the gathered patches in F, both free
+        // until the first block
+        int32_t *src_row = static_cast<int32_t *>(h->QKV);
+        ProfScope ps(h, s, P_POS);
+        VIT_TRY(vith::window_positions_launch(grid, n_images, P, d.patch_order, window, h->pos, h->merge_row,
+                                              src_row, s));
+        ++nl;
+        VIT_TRY(vith::gather_rows_launch(patches, src_row, h->F, P, VIT_PATCH_DIM * 2, s));
+        ++nl;
+        patches = h->F;
     }
 
-    CUtensorMap mPatch, mH, mF, mH4, mF4;
+    CUtensorMap mPatch, mH, mF, mH4, mF4, mWin;
     vith::AttnMaps mQKV;
     VIT_TRY(vith::gemm_make_a_map(&mPatch, patches, P, VIT_PATCH_DIM));
+    if (window > 0 && window <= 8) VIT_TRY(vith::win_make_map(&mWin, h->QKV, P));
     VIT_TRY(vith::gemm_make_a_map(&mH, h->H, P, VIT_WIDTH));
     VIT_TRY(vith::gemm_make_a_map(&mF, h->F, P, VIT_MLP));
     VIT_TRY(vith::gemm_make_a_map(&mH4, h->H, M4, VIT_MERGE_DIM));
@@ -258,9 +276,17 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
                                       h->pos, h->rope_cs, h->status, s));
             ++nl;
         }
-        {
+        if (window == 0 || h->full_attention[l]) {
             ProfScope ps(h, s, P_ATT);
             VIT_TRY(vith::attn_launch(mQKV, cu.data(), n_seg, h->H, h->status, s));
+            ++nl;
+        } else if (window <= 8) {
+            ProfScope ps(h, s, P_WATT);
+            VIT_TRY(vith::win_attn_launch(mWin, grid, n_images, window, h->H, h->status, s));
+            ++nl;
+        } else {
+            ProfScope ps(h, s, P_WATT);
+            VIT_TRY(vith::attn_launch(mQKV, cu_win.data(), static_cast<int>(cu_win.size()) - 1, h->H, h->status, s));
             ++nl;
         }
         {
@@ -290,7 +316,7 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
     {
         ProfScope ps(h, s, P_LN);
         VIT_TRY(vith::layernorm_launch(h->X, d.lnq_w, d.lnq_b, h->H, P, d.ln_eps,
-                                       d.patch_order == 1 ? h->merge_row : nullptr, s));
+                                       (d.patch_order == 1 || window > 0) ? h->merge_row : nullptr, s));
         ++nl;
     }
     {
@@ -416,6 +442,7 @@ int vit_weights_create(const vit_weights_desc *d, vit_handle **out) {
     if (d->depth < 1 || d->depth > 64 || d->out_dim < 16 || d->out_dim > 16384 || (d->out_dim % 16) != 0 ||
         !(d->ln_eps > 0.0f) || (d->patch_order != 0 && d->patch_order != 1) || !d->layers)
         return VIT_ERR_ARG;
+    if (d->window < 0 || d->window > VIT_MAX_SIDE || (d->window % 2) != 0) return VIT_ERR_ARG;
     const void *req[] = {d->pe_w, d->lnq_w, d->m0_w, d->m2_w};
     for (const void *p : req)
         if (!p) return VIT_ERR_ARG;
@@ -439,6 +466,10 @@ int vit_weights_create(const vit_weights_desc *d, vit_handle **out) {
     h->desc = *d;
     h->layers.assign(d->layers, d->layers + d->depth);
     h->desc.layers = nullptr;
+    h->full_attention.assign(d->depth, 0);
+    if (d->window > 0 && d->full_attention)
+        for (int l = 0; l < d->depth; ++l) h->full_attention[l] = d->full_attention[l] ? 1 : 0;
+    h->desc.full_attention = nullptr;
     cudaGetDevice(&h->device);
     h->maps.resize(d->depth);
     rc = vith::gemm_make_b_map(&h->pe_map, d->pe_w, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32);
@@ -619,6 +650,36 @@ int vit_op_attention(const void *qkv, int64_t P, const int32_t *cu_seqlens, int 
     const int rc = vith::attn_make_maps(&t, qkv, P);
     if (rc != VIT_OK) return rc;
     return vith::attn_launch(t, cu_seqlens, n_seg, out, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+int vit_op_window_positions(const int32_t *grid_thw, int n_images, int patch_order, int window, int32_t *pos,
+                            int32_t *merge_row, int32_t *src_row, void *stream) {
+    if (!pos || !merge_row || !src_row || (patch_order != 0 && patch_order != 1)) return VIT_ERR_ARG;
+    if (window < 2 || window > VIT_MAX_SIDE || window % 2) return VIT_ERR_ARG;
+    int64_t P = 0;
+    const int rc = validate_grids(grid_thw, n_images, VIT_MAX_IMAGES, &P);
+    if (rc != VIT_OK) return rc;
+    return vith::window_positions_launch(grid_thw, n_images, P, patch_order, window, pos, merge_row, src_row,
+                                         static_cast<cudaStream_t>(stream));
+}
+
+int vit_op_gather_rows(const void *src, const int32_t *src_row, void *dst, int64_t rows, int row_bytes,
+                       void *stream) {
+    if (!src || !src_row || !dst || rows < 0 || row_bytes <= 0) return VIT_ERR_ARG;
+    return vith::gather_rows_launch(src, src_row, dst, rows, row_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int vit_op_window_attention(const void *qkv, const int32_t *grid_thw, int n_images, int window, void *out,
+                            int32_t *dev_status, void *stream) {
+    if (!qkv || !out || window < 2 || window > 8 || window % 2) return VIT_ERR_ARG;
+    int64_t P = 0;
+    int rc = validate_grids(grid_thw, n_images, VIT_MAX_IMAGES, &P);
+    if (rc != VIT_OK) return rc;
+    if (!aligned16(qkv) || !aligned16(out)) return VIT_ERR_ALIGN;
+    CUtensorMap m;
+    rc = vith::win_make_map(&m, qkv, P);
+    if (rc != VIT_OK) return rc;
+    return vith::win_attn_launch(m, grid_thw, n_images, window, out, dev_status, static_cast<cudaStream_t>(stream));
 }
 
 int vit_op_wait_selftest(int32_t *dev_status, int64_t limit_cycles, void *stream) {

@@ -13,12 +13,13 @@ namespace vith {
 struct LayerMaps {
     CUtensorMap qkv, proj, fc1, fc2;
 };
-constexpr int kProfClasses = 10;
+constexpr int kProfClasses = 11;
 }  // namespace vith
 
 struct vit_handle {
     vit_weights_desc desc{};
     std::vector<vit_layer_w> layers;
+    std::vector<uint8_t> full_attention;   // [depth], windowed handles only
     std::vector<vith::LayerMaps> maps;
     CUtensorMap pe_map{}, m0_map{}, m2_map{};
     int device = 0;
@@ -29,8 +30,9 @@ struct vit_handle {
     int64_t ws_patches = 0;
     float *X = nullptr;            // fp32 [P, 1280] residual stream
     void *H = nullptr;             // bf16 [P, 1280] LayerNorm output / attention output / merger input
-    void *QKV = nullptr;           // bf16 [P, 3840]
-    void *F = nullptr;             // bf16 [P, 5120] fc1 output / merger hidden
+    void *QKV = nullptr;           // bf16 [P, 3840]; with windows, first the gather's source rows
+    void *F = nullptr;             // bf16 [P, 5120] fc1 output / merger hidden; with windows, first
+                                   // the patches gathered into window order (bf16 [P, 1176])
     int32_t *pos = nullptr;        // [P]
     int32_t *merge_row = nullptr;  // [P]
     void *patch_stage = nullptr;   // bf16 [P, 1176] (vit_encode_host)

@@ -4,6 +4,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <vector>
+
 #include "../../include/vit.h"
 #include "../../include/vit_ops.h"
 
@@ -47,6 +49,16 @@ int attn_launch_stack(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg
                       cudaStream_t s);
 int positions_launch_stack(const int32_t *grid_thw, int n_images, int64_t P, int patch_order, int32_t *pos,
                            int32_t *merge_row, cudaStream_t s);
+// ---- windowed attention (window.cu); window = side in patches (even)
+int window_cu_seqlens(const int32_t *grid_thw, int n_images, int window, std::vector<int32_t> &cu);
+int window_positions_launch(const int32_t *grid_thw, int n_images, int64_t P, int patch_order, int window,
+                            int32_t *pos, int32_t *merge_row, int32_t *src_row, cudaStream_t s);
+int gather_rows_launch(const void *src, const int32_t *src_row, void *dst, int64_t rows, int row_bytes,
+                       cudaStream_t s);
+int win_make_map(CUtensorMap *m, const void *qkv, int64_t P);
+// window <= 8; the windows are derived from the grids on the device
+int win_attn_launch(const CUtensorMap &tm, const int32_t *grid_thw, int n_images, int window, void *out,
+                    int32_t *status, cudaStream_t s);
 int wait_selftest_launch(int32_t *status, long long limit, cudaStream_t s);
 int mrope_launch(const int32_t *ids, int64_t L, const int32_t *grid_thw, int n_grids, int32_t *out, int32_t *delta,
                  int32_t *status, cudaStream_t s);

@@ -34,7 +34,11 @@ class VitWeightsDesc(ctypes.Structure):
     _fields_ = [("depth", c_int), ("out_dim", c_int), ("ln_eps", c_float), ("patch_order", c_int),
                 ("pe_w", c_void_p), ("pe_b", c_void_p), ("layers", ctypes.POINTER(VitLayerW)),
                 ("lnq_w", c_void_p), ("lnq_b", c_void_p), ("m0_w", c_void_p), ("m0_b", c_void_p),
-                ("m2_w", c_void_p), ("m2_b", c_void_p)]
+                ("m2_w", c_void_p), ("m2_b", c_void_p), ("window", c_int),
+                ("full_attention", ctypes.POINTER(ctypes.c_uint8))]
+
+# The Qwen2.5-VL tower's full-attention blocks (0-based) when windows are on
+QWEN25_FULL_BLOCKS = (7, 15, 23, 31)
 
 
 _SIGS = {
@@ -60,6 +64,9 @@ _SIGS = {
     "vit_op_layernorm": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_float, c_void_p, c_void_p]),
     "vit_op_attention": (c_int, [c_void_p, c_int64, c_i32p, c_int, c_void_p, c_void_p, c_void_p]),
     "vit_op_wait_selftest": (c_int, [c_void_p, c_int64, c_void_p]),
+    "vit_op_window_positions": (c_int, [c_i32p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "vit_op_gather_rows": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int, c_void_p]),
+    "vit_op_window_attention": (c_int, [c_void_p, c_i32p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
 }
 
 _lib = None
@@ -159,9 +166,12 @@ def random_weights_device(depth: int, out_dim: int, seed: int, device="cuda", st
 
 
 class VisionEncoder:
-    """A validated weight view (vit_handle) and its workspace; ``encode`` runs vit_encode."""
+    """A validated weight view (vit_handle) and its workspace; ``encode`` runs vit_encode.
+    window > 0 makes the windowed (Qwen2.5-VL) tower: blocks in ``full_blocks`` attend over the
+    whole frame, the others inside window x window patches."""
 
-    def __init__(self, weights: Dict, out_dim: int, eps: float = 1e-6, patch_order: int = 0):
+    def __init__(self, weights: Dict, out_dim: int, eps: float = 1e-6, patch_order: int = 0, window: int = 0,
+                 full_blocks: Sequence[int] = ()):
         self.weights = weights          # keeps the device tensors alive
         self.out_dim = out_dim
         depth = len(weights["layers"])
@@ -175,6 +185,9 @@ class VisionEncoder:
         d.layers = self._layers
         for k in ("lnq_w", "lnq_b", "m0_w", "m0_b", "m2_w", "m2_b"):
             setattr(d, k, _ptr(weights.get(k)))
+        d.window = int(window)
+        self._full = (ctypes.c_uint8 * depth)(*[1 if l in set(full_blocks) else 0 for l in range(depth)])
+        d.full_attention = ctypes.cast(self._full, ctypes.POINTER(ctypes.c_uint8))
         self._desc = d
         h = c_void_p()
         check(lib().vit_weights_create(ctypes.byref(d), ctypes.byref(h)), "vit_weights_create")
@@ -286,6 +299,30 @@ def op_attention(qkv, cu_seqlens: Sequence[int], out, status=None, stream=None):
     cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
     check(lib().vit_op_attention(_ptr(qkv), qkv.shape[0], cu.ctypes.data_as(c_i32p), cu.shape[0] - 1, _ptr(out),
                                  _ptr(status), _stream(stream)), "vit_op_attention")
+    return out
+
+
+def op_window_positions(grid_thw, patch_order: int, window: int, device="cuda", stream=None):
+    """(pos, merge_row, src_row) of the window-order rows, int32 [P] each."""
+    g = _grid_arg(grid_thw)
+    P, _ = encode_sizes(g)
+    pos, mr, src = (torch.empty(P, dtype=torch.int32, device=device) for _ in range(3))
+    check(lib().vit_op_window_positions(_gp(g), g.shape[0], patch_order, window, _ptr(pos), _ptr(mr), _ptr(src),
+                                        _stream(stream)), "vit_op_window_positions")
+    return pos, mr, src
+
+
+def op_gather_rows(src, src_row, dst, stream=None):
+    row_bytes = src.shape[1] * src.element_size()
+    check(lib().vit_op_gather_rows(_ptr(src), _ptr(src_row), _ptr(dst), dst.shape[0], row_bytes, _stream(stream)),
+          "vit_op_gather_rows")
+    return dst
+
+
+def op_window_attention(qkv, grid_thw, window: int, out, status=None, stream=None):
+    g = _grid_arg(grid_thw)
+    check(lib().vit_op_window_attention(_ptr(qkv), _gp(g), g.shape[0], window, _ptr(out), _ptr(status),
+                                        _stream(stream)), "vit_op_window_attention")
     return out
 
 

@@ -78,6 +78,24 @@ def test_weights_create_rejects_bad_descriptors_before_cuda(lib):
         setattr(layers[0], k, fake)
     layers[0].qkv_w = fake + 2
     assert lib.vit_weights_create(ctypes.byref(d), ctypes.byref(h)) == nv.VIT_ERR_ALIGN
+    layers[0].qkv_w = fake
+    for bad_window in (-2, 7, 8194):                      # windows: even, 2 .. max side
+        d.window = bad_window
+        assert lib.vit_weights_create(ctypes.byref(d), ctypes.byref(h)) == nv.VIT_ERR_ARG
+
+
+def test_window_ops_reject_bad_arguments_before_cuda(lib):
+    from resolution_vit_vision_b200 import native as nv
+    g = np.array([[1, 8, 8]], np.int32)
+    p = ctypes.c_void_p(0x10000)
+    for w in (0, 3, 10):                                  # the window kernel takes sides 2, 4, 6, 8
+        assert lib.vit_op_window_attention(p, nv._gp(g), 1, w, p, None, None) == nv.VIT_ERR_ARG
+    assert lib.vit_op_window_attention(ctypes.c_void_p(0x10002), nv._gp(g), 1, 8, p, None, None) == nv.VIT_ERR_ALIGN
+    bad = np.array([[1, 7, 8]], np.int32)
+    assert lib.vit_op_window_attention(p, nv._gp(bad), 1, 8, p, None, None) == nv.VIT_ERR_GRID
+    assert lib.vit_op_window_positions(nv._gp(g), 1, 0, 5, p, p, p, None) == nv.VIT_ERR_ARG
+    assert lib.vit_op_window_positions(nv._gp(g), 1, 2, 8, p, p, p, None) == nv.VIT_ERR_ARG
+    assert lib.vit_op_gather_rows(p, p, p, 4, 2352 + 8, None) == nv.VIT_ERR_ALIGN
 
 
 def test_mrope_rejects_bad_arguments(lib):
