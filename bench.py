@@ -46,6 +46,8 @@ def parse():
                     help="the windowed (Qwen2.5-VL) tower: window side in patches (8 = 112 px); 0 = Qwen2-VL")
     ap.add_argument("--full-blocks", default="7,15,23,31",
                     help="with --window: the full-attention blocks (0-based, comma-separated)")
+    ap.add_argument("--op", default=None, choices=["mrope_apply", "scatter"],
+                    help="time one decoder-side step on the prompt that carries the workload's merged tokens")
     return ap.parse_args()
 
 
@@ -234,11 +236,70 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------------------ decoder-side steps
+def run_op(args):
+    """One decoder-side step (HBM-bound) on the prefill prompt that carries the workload's merged
+    tokens: 3-D M-RoPE on q [L, 28, 128] and k [L, 4, 128], or the scatter of the merged tokens into
+    the [L, 3584] input sequence with a 152064-row embedding table."""
+    import torch
+    from resolution_vit_vision_b200 import native as nv
+    from resolution_vit_vision_b200 import synthetic as syn
+    wl = syn.WORKLOADS[args.workload]
+    ids, grids = syn.decoder_prompt(wl.grids, wl.seed)
+    L = int(ids.size)
+    dev = torch.device("cuda", 0)
+    t_ids = torch.from_numpy(ids.astype(np.int32)).to(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.seed)
+    if args.op == "mrope_apply":
+        pos, _ = nv.mrope_index(t_ids, grids)
+        q = torch.randn((L, 28, 128), generator=g, device=dev).to(torch.bfloat16)
+        k = torch.randn((L, 4, 128), generator=g, device=dev).to(torch.bfloat16)
+        step = lambda: nv.mrope_apply(q, k, pos)
+        nbytes = 2 * (q.numel() + k.numel()) * 2 + pos.numel() * 4
+        unit_desc = "q [L, 28, 128] and k [L, 4, 128] read and written once, ids read"
+    else:
+        n_vis = sum(t * h * w // 4 for t, h, w in grids)
+        table = torch.randn((152064, 3584), generator=g, device=dev).to(torch.bfloat16)
+        vision = torch.randn((n_vis, 3584), generator=g, device=dev).to(torch.bfloat16)
+        out = torch.empty((L, 3584), dtype=torch.bfloat16, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        step = lambda: nv.scatter_vision_tokens(t_ids, table, vision, out=out, status=st)
+        nbytes = 2 * L * 3584 * 2 + L * 4
+        unit_desc = "every output row read once (table or vision) and written once, ids read"
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    stream = torch.cuda.current_stream()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if args.op == "scatter":
+        assert int(st.item()) == 0
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    pk, pk_kind = peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    print(json.dumps({"op": args.op, "metric": f"{args.op} GB/s (algorithmic bytes)", "value": gbs, "unit": "GB/s",
+                      "ms_per_step": ms, "steps": args.steps, "tokens": L, "bytes": nbytes, "bytes_are": unit_desc,
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                   "frac": gbs / pk["hbm_gbs"], "peak_source": f"{pk_kind} hbm_gbs"},
+                      "config": {"workload": f"prefill prompt carrying the {wl.name} batch's merged tokens",
+                                 "L": L, "l2": "flushed between steps (256 MB write)"}}), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------------------ native arm
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op:
+        return run_op(args)
     import torch
     import torch.distributed as dist
 

@@ -69,21 +69,25 @@ int vit_op_attention(const void *qkv, int64_t P, const int32_t *cu_seqlens, int 
  * over the windows of window x window patches (window even, >= 2) in raster order, inside a window
  * over its 2x2 merge groups in raster order, inside a group (dh, dw). For each window-order row r:
  * pos[r] = (h << 16) | w inside its frame, src_row[r] = the row holding that patch when the images
- * are packed in patch_order (0 block, 1 raster), merge_row[r] = its row in 2x2-block order. All
- * three are int32 [P] device buffers (required). grid_thw: HOST [n_images, 3]. */
+ * are packed in patch_order (0 block, 1 raster), merge_row[r] = its row in 2x2-block order (int32
+ * [P] device buffers each). win_table: int32 [2 * n_windows] device (n_windows <= P / 4), receives
+ * (first row, number of rows) of every window in window order; *n_windows (HOST int) receives the
+ * number of windows. All outputs required. grid_thw: HOST [n_images, 3]. */
 int vit_op_window_positions(const int32_t *grid_thw, int n_images, int patch_order, int window, int32_t *pos,
-                            int32_t *merge_row, int32_t *src_row, void *stream);
+                            int32_t *merge_row, int32_t *src_row, int32_t *win_table, int *n_windows,
+                            void *stream);
 
 /* dst[r, :] = src[src_row[r], :] for rows of row_bytes bytes (a multiple of 16; src, dst
  * 16-byte aligned). src_row: int32 [rows] device, each in range of src (not checked). */
 int vit_op_gather_rows(const void *src, const int32_t *src_row, void *dst, int64_t rows, int row_bytes,
                        void *stream);
 
-/* Attention inside windows (same architecture note): qkv bf16 [P, 3840] with its rows in window
- * order for the images of grid_thw (HOST [n_images, 3]); every window of window x window patches
- * (window even, 2..8) is one segment, attended exactly as by vit_op_attention. out: bf16 [P, 1280]
- * in the same row order. dev_status as for vit_op_attention. */
-int vit_op_window_attention(const void *qkv, const int32_t *grid_thw, int n_images, int window, void *out,
+/* Attention inside windows (same architecture note): qkv bf16 [P, 3840]; win_table: int32
+ * [2 * n_windows] device, (first row, rows) of each window as vit_op_window_positions writes it
+ * (windows of at most 8 x 8 patches: rows <= 64; the table is trusted, the kernel only keeps its
+ * stores below row P). Every window is one segment, attended exactly as by vit_op_attention.
+ * out: bf16 [P, 1280], same row order. dev_status as for vit_op_attention. */
+int vit_op_window_attention(const void *qkv, int64_t P, const int32_t *win_table, int n_windows, void *out,
                             int32_t *dev_status, void *stream);
 
 /* Bounded-wait self-test (the failure path of every tensor-core kernel's mbarrier waits, run on

@@ -155,6 +155,7 @@ int ensure_workspace(vit_handle *h, int64_t P) {
     const size_t oF = take(static_cast<size_t>(Pn) * VIT_MLP * 2);
     const size_t oPos = take(static_cast<size_t>(Pn) * 4);
     const size_t oMr = take(static_cast<size_t>(Pn) * 4);
+    const size_t oWt = take(static_cast<size_t>(Pn / 4 + 1) * 8);
     const size_t oPs = take(static_cast<size_t>(Pn) * VIT_PATCH_DIM * 2);
     const size_t oOs = take(static_cast<size_t>(Pn / 4 + 1) * out_dim * 2);
     const size_t oCs = take(static_cast<size_t>(VIT_MAX_SIDE) * 40 * 4);
@@ -181,6 +182,7 @@ int ensure_workspace(vit_handle *h, int64_t P) {
     h->F = b + oF;
     h->pos = reinterpret_cast<int32_t *>(b + oPos);
     h->merge_row = reinterpret_cast<int32_t *>(b + oMr);
+    h->win_tab = reinterpret_cast<int32_t *>(b + oWt);
     h->patch_stage = b + oPs;
     h->out_stage = b + oOs;
     h->rope_cs = reinterpret_cast<float *>(b + oCs);
@@ -233,17 +235,19 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
         int32_t *src_row = static_cast<int32_t *>(h->QKV);
         ProfScope ps(h, s, P_POS);
         VIT_TRY(vith::window_positions_launch(grid, n_images, P, d.patch_order, window, h->pos, h->merge_row,
-                                              src_row, s));
+                                              src_row, h->win_tab, s));
         ++nl;
         VIT_TRY(vith::gather_rows_launch(patches, src_row, h->F, P, VIT_PATCH_DIM * 2, s));
         ++nl;
         patches = h->F;
     }
 
-    CUtensorMap mPatch, mH, mF, mH4, mF4, mWin;
+    CUtensorMap mPatch, mH, mF, mH4, mF4;
+    vith::WinMaps mWin;
+    const int n_windows = window > 0 ? vith::window_count(grid, n_images, window) : 0;
     vith::AttnMaps mQKV;
     VIT_TRY(vith::gemm_make_a_map(&mPatch, patches, P, VIT_PATCH_DIM));
-    if (window > 0 && window <= 8) VIT_TRY(vith::win_make_map(&mWin, h->QKV, P));
+    if (window > 0 && window <= 8) VIT_TRY(vith::win_make_maps(&mWin, h->QKV, P));
     VIT_TRY(vith::gemm_make_a_map(&mH, h->H, P, VIT_WIDTH));
     VIT_TRY(vith::gemm_make_a_map(&mF, h->F, P, VIT_MLP));
     VIT_TRY(vith::gemm_make_a_map(&mH4, h->H, M4, VIT_MERGE_DIM));
@@ -282,7 +286,7 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
             ++nl;
         } else if (window <= 8) {
             ProfScope ps(h, s, P_WATT);
-            VIT_TRY(vith::win_attn_launch(mWin, grid, n_images, window, h->H, h->status, s));
+            VIT_TRY(vith::win_attn_launch(mWin, h->win_tab, n_windows, P, h->H, h->status, s));
             ++nl;
         } else {
             ProfScope ps(h, s, P_WATT);
@@ -653,14 +657,17 @@ int vit_op_attention(const void *qkv, int64_t P, const int32_t *cu_seqlens, int 
 }
 
 int vit_op_window_positions(const int32_t *grid_thw, int n_images, int patch_order, int window, int32_t *pos,
-                            int32_t *merge_row, int32_t *src_row, void *stream) {
-    if (!pos || !merge_row || !src_row || (patch_order != 0 && patch_order != 1)) return VIT_ERR_ARG;
+                            int32_t *merge_row, int32_t *src_row, int32_t *win_table, int *n_windows,
+                            void *stream) {
+    if (!pos || !merge_row || !src_row || !win_table || !n_windows || (patch_order != 0 && patch_order != 1))
+        return VIT_ERR_ARG;
     if (window < 2 || window > VIT_MAX_SIDE || window % 2) return VIT_ERR_ARG;
     int64_t P = 0;
     const int rc = validate_grids(grid_thw, n_images, VIT_MAX_IMAGES, &P);
     if (rc != VIT_OK) return rc;
+    *n_windows = vith::window_count(grid_thw, n_images, window);
     return vith::window_positions_launch(grid_thw, n_images, P, patch_order, window, pos, merge_row, src_row,
-                                         static_cast<cudaStream_t>(stream));
+                                         win_table, static_cast<cudaStream_t>(stream));
 }
 
 int vit_op_gather_rows(const void *src, const int32_t *src_row, void *dst, int64_t rows, int row_bytes,
@@ -669,17 +676,39 @@ int vit_op_gather_rows(const void *src, const int32_t *src_row, void *dst, int64
     return vith::gather_rows_launch(src, src_row, dst, rows, row_bytes, static_cast<cudaStream_t>(stream));
 }
 
-int vit_op_window_attention(const void *qkv, const int32_t *grid_thw, int n_images, int window, void *out,
+int vit_op_window_attention(const void *qkv, int64_t P, const int32_t *win_table, int n_windows, void *out,
                             int32_t *dev_status, void *stream) {
-    if (!qkv || !out || window < 2 || window > 8 || window % 2) return VIT_ERR_ARG;
-    int64_t P = 0;
-    int rc = validate_grids(grid_thw, n_images, VIT_MAX_IMAGES, &P);
-    if (rc != VIT_OK) return rc;
+    if (!qkv || !out || !win_table || P < 1 || n_windows < 1 || n_windows > P / 4) return VIT_ERR_ARG;
+    if (P > VIT_MAX_PATCHES) return VIT_ERR_LIMIT;
     if (!aligned16(qkv) || !aligned16(out)) return VIT_ERR_ALIGN;
-    CUtensorMap m;
-    rc = vith::win_make_map(&m, qkv, P);
+    vith::WinMaps m;
+    const int rc = vith::win_make_maps(&m, qkv, P);
     if (rc != VIT_OK) return rc;
-    return vith::win_attn_launch(m, grid_thw, n_images, window, out, dev_status, static_cast<cudaStream_t>(stream));
+    return vith::win_attn_launch(m, win_table, n_windows, P, out, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+int mrope_apply(void *q, int n_heads, void *k, int n_kv_heads, int head_dim, const int32_t *pos, int64_t L,
+                double theta, const int32_t *sections, void *stream) {
+    if (!pos || !sections || L < 0 || L > (int64_t(1) << 31) - 1 || !(theta > 1.0)) return VIT_ERR_ARG;
+    if (head_dim < 16 || head_dim > 256 || head_dim % 16) return VIT_ERR_ARG;
+    if (n_heads < 0 || n_kv_heads < 0 || (n_heads > 0 && !q) || (n_kv_heads > 0 && !k)) return VIT_ERR_ARG;
+    if (n_heads * head_dim > 65536 || n_kv_heads * head_dim > 65536) return VIT_ERR_ARG;
+    if (sections[0] < 0 || sections[1] < 0 || sections[2] < 0 || sections[0] + sections[1] + sections[2] != head_dim / 2)
+        return VIT_ERR_ARG;
+    if ((q && !aligned16(q)) || (k && !aligned16(k))) return VIT_ERR_ALIGN;
+    return vith::mrope_apply_launch(n_heads > 0 ? q : nullptr, n_heads, n_kv_heads > 0 ? k : nullptr, n_kv_heads,
+                                    head_dim, pos, L, theta, sections, static_cast<cudaStream_t>(stream));
+}
+
+int scatter_vision_tokens(const int32_t *input_ids, int64_t L, const void *embed_table, int64_t vocab, int dim,
+                          const void *vision, int64_t n_vision, void *out, int32_t *dev_status, void *stream) {
+    if (L == 0 && n_vision == 0) return VIT_OK;   // an empty prompt: nothing to read or write
+    if (!input_ids || !embed_table || !out || L < 0 || L > (int64_t(1) << 18) || vocab < 1 || dim < 8 ||
+        dim % 8 || n_vision < 0 || (n_vision > 0 && !vision))
+        return VIT_ERR_ARG;
+    if (!aligned16(embed_table) || !aligned16(out) || (vision && !aligned16(vision))) return VIT_ERR_ALIGN;
+    return vith::scatter_launch(input_ids, L, embed_table, vocab, dim, vision, n_vision, out, dev_status,
+                                static_cast<cudaStream_t>(stream));
 }
 
 int vit_op_wait_selftest(int32_t *dev_status, int64_t limit_cycles, void *stream) {

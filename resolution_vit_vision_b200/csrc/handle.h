@@ -35,6 +35,7 @@ struct vit_handle {
                                    // the patches gathered into window order (bf16 [P, 1176])
     int32_t *pos = nullptr;        // [P]
     int32_t *merge_row = nullptr;  // [P]
+    int32_t *win_tab = nullptr;    // [2 * (P/4 + 1)] (first row, rows) per attention window
     void *patch_stage = nullptr;   // bf16 [P, 1176] (vit_encode_host)
     void *out_stage = nullptr;     // bf16 [P/4, out_dim] (vit_encode_host)
     float *rope_cs = nullptr;      // [VIT_MAX_SIDE][20][2]

@@ -7,6 +7,7 @@
 #include <vector>
 
 #include "../../include/vit.h"
+#include "../../include/vit_decoder.h"
 #include "../../include/vit_ops.h"
 
 namespace vith {
@@ -51,14 +52,24 @@ int positions_launch_stack(const int32_t *grid_thw, int n_images, int64_t P, int
                            int32_t *merge_row, cudaStream_t s);
 // ---- windowed attention (window.cu); window = side in patches (even)
 int window_cu_seqlens(const int32_t *grid_thw, int n_images, int window, std::vector<int32_t> &cu);
+int window_count(const int32_t *grid_thw, int n_images, int window);
+// win_tab: int32 [2 * window_count] device, receives (first row, rows) per window
 int window_positions_launch(const int32_t *grid_thw, int n_images, int64_t P, int patch_order, int window,
-                            int32_t *pos, int32_t *merge_row, int32_t *src_row, cudaStream_t s);
+                            int32_t *pos, int32_t *merge_row, int32_t *src_row, int32_t *win_tab, cudaStream_t s);
 int gather_rows_launch(const void *src, const int32_t *src_row, void *dst, int64_t rows, int row_bytes,
                        cudaStream_t s);
-int win_make_map(CUtensorMap *m, const void *qkv, int64_t P);
-// window <= 8; the windows are derived from the grids on the device
-int win_attn_launch(const CUtensorMap &tm, const int32_t *grid_thw, int n_images, int window, void *out,
-                    int32_t *status, cudaStream_t s);
+struct WinMaps {
+    CUtensorMap m32, m128;
+};
+int win_make_maps(WinMaps *m, const void *qkv, int64_t P);
+// windows of at most 64 rows, from the table window_positions_launch wrote
+int win_attn_launch(const WinMaps &m, const int32_t *win_tab, int n_windows, int64_t P, void *out, int32_t *status,
+                    cudaStream_t s);
+// ---- decoder-side steps (decoder.cu)
+int mrope_apply_launch(void *q, int Hq, void *k, int Hk, int D, const int32_t *pos, int64_t L, double theta,
+                       const int32_t *sections, cudaStream_t s);
+int scatter_launch(const int32_t *ids, int64_t L, const void *table, int64_t vocab, int dim, const void *vision,
+                   int64_t n_vision, void *out, int32_t *status, cudaStream_t s);
 int wait_selftest_launch(int32_t *status, long long limit, cudaStream_t s);
 int mrope_launch(const int32_t *ids, int64_t L, const int32_t *grid_thw, int n_grids, int32_t *out, int32_t *delta,
                  int32_t *status, cudaStream_t s);

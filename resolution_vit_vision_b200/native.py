@@ -64,9 +64,14 @@ _SIGS = {
     "vit_op_layernorm": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_float, c_void_p, c_void_p]),
     "vit_op_attention": (c_int, [c_void_p, c_int64, c_i32p, c_int, c_void_p, c_void_p, c_void_p]),
     "vit_op_wait_selftest": (c_int, [c_void_p, c_int64, c_void_p]),
-    "vit_op_window_positions": (c_int, [c_i32p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "mrope_apply": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_int64, ctypes.c_double, c_i32p,
+                            c_void_p]),
+    "scatter_vision_tokens": (c_int, [c_void_p, c_int64, c_void_p, c_int64, c_int, c_void_p, c_int64, c_void_p,
+                                      c_void_p, c_void_p]),
+    "vit_op_window_positions": (c_int, [c_i32p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                        ctypes.POINTER(c_int), c_void_p]),
     "vit_op_gather_rows": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int, c_void_p]),
-    "vit_op_window_attention": (c_int, [c_void_p, c_i32p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "vit_op_window_attention": (c_int, [c_void_p, c_int64, c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
 }
 
 _lib = None
@@ -303,13 +308,16 @@ def op_attention(qkv, cu_seqlens: Sequence[int], out, status=None, stream=None):
 
 
 def op_window_positions(grid_thw, patch_order: int, window: int, device="cuda", stream=None):
-    """(pos, merge_row, src_row) of the window-order rows, int32 [P] each."""
+    """(pos, merge_row, src_row) of the window-order rows, int32 [P] each, and the window table
+    int32 [n_windows, 2] = (first row, rows)."""
     g = _grid_arg(grid_thw)
     P, _ = encode_sizes(g)
     pos, mr, src = (torch.empty(P, dtype=torch.int32, device=device) for _ in range(3))
+    tab = torch.empty((P // 4 + 1, 2), dtype=torch.int32, device=device)
+    n = c_int(0)
     check(lib().vit_op_window_positions(_gp(g), g.shape[0], patch_order, window, _ptr(pos), _ptr(mr), _ptr(src),
-                                        _stream(stream)), "vit_op_window_positions")
-    return pos, mr, src
+                                        _ptr(tab), ctypes.byref(n), _stream(stream)), "vit_op_window_positions")
+    return pos, mr, src, tab[:n.value]
 
 
 def op_gather_rows(src, src_row, dst, stream=None):
@@ -319,10 +327,36 @@ def op_gather_rows(src, src_row, dst, stream=None):
     return dst
 
 
-def op_window_attention(qkv, grid_thw, window: int, out, status=None, stream=None):
-    g = _grid_arg(grid_thw)
-    check(lib().vit_op_window_attention(_ptr(qkv), _gp(g), g.shape[0], window, _ptr(out), _ptr(status),
-                                        _stream(stream)), "vit_op_window_attention")
+def op_window_attention(qkv, win_table, out, status=None, stream=None):
+    """win_table: int32 [n_windows, 2] device (first row, rows), as op_window_positions returns."""
+    check(lib().vit_op_window_attention(_ptr(qkv), qkv.shape[0], _ptr(win_table), win_table.shape[0], _ptr(out),
+                                        _ptr(status), _stream(stream)), "vit_op_window_attention")
+    return out
+
+
+MROPE_THETA = 1.0e6
+MROPE_SECTIONS = (16, 24, 24)
+
+
+def mrope_apply(q, k, pos, theta: float = MROPE_THETA, sections=MROPE_SECTIONS, stream=None):
+    """3-D M-RoPE in place on q [L, heads, head_dim] and k [L, kv_heads, head_dim] (bf16, either may
+    be None); pos int32 [3, L] from mrope_index."""
+    x = q if q is not None else k
+    L, D = x.shape[0], x.shape[2]
+    sec = np.ascontiguousarray(np.asarray(sections, dtype=np.int32))
+    check(lib().mrope_apply(_ptr(q), 0 if q is None else q.shape[1], _ptr(k), 0 if k is None else k.shape[1], D,
+                            _ptr(pos), L, float(theta), sec.ctypes.data_as(c_i32p), _stream(stream)), "mrope_apply")
+    return q, k
+
+
+def scatter_vision_tokens(input_ids, embed_table, vision, out=None, status=None, stream=None):
+    """The decoder's input rows: vision tokens at the image / video placeholders, embeddings elsewhere."""
+    L, (V, D) = input_ids.shape[0], embed_table.shape
+    if out is None:
+        out = torch.empty((L, D), dtype=embed_table.dtype, device=embed_table.device)
+    n_vis = 0 if vision is None else vision.shape[0]
+    check(lib().scatter_vision_tokens(_ptr(input_ids), L, _ptr(embed_table), V, D, _ptr(vision), n_vis, _ptr(out),
+                                      _ptr(status), _stream(stream)), "scatter_vision_tokens")
     return out
 
 

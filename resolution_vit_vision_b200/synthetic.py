@@ -189,6 +189,15 @@ def make_prompt(segments, seed: int) -> np.ndarray:
     return np.concatenate(out) if out else np.zeros((0,), np.int32)
 
 
+def decoder_prompt(grids, seed: int, text_between: int = 300) -> Tuple[np.ndarray, np.ndarray]:
+    """A prefill prompt that carries a whole encoded batch: text, then each image's merged tokens
+    (t*h*w/4 image tokens) followed by ``text_between`` text tokens."""
+    segs = [("text", 512)]
+    for t, h, w in grids:
+        segs += [("image", t * h * w // 4), ("text", text_between)]
+    return make_prompt(segs, seed), np.asarray(grids, np.int32).reshape(-1, 3)
+
+
 def tiny_prompt(seed: int = 0) -> Tuple[np.ndarray, np.ndarray]:
     """[8 text][vision_start][16 image tokens][vision_end][8 text] with grid (1,8,8)."""
     ids = make_prompt([("text", 8), ("image", 16), ("text", 8)], seed)

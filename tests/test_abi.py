@@ -88,13 +88,18 @@ def test_window_ops_reject_bad_arguments_before_cuda(lib):
     from resolution_vit_vision_b200 import native as nv
     g = np.array([[1, 8, 8]], np.int32)
     p = ctypes.c_void_p(0x10000)
-    for w in (0, 3, 10):                                  # the window kernel takes sides 2, 4, 6, 8
-        assert lib.vit_op_window_attention(p, nv._gp(g), 1, w, p, None, None) == nv.VIT_ERR_ARG
-    assert lib.vit_op_window_attention(ctypes.c_void_p(0x10002), nv._gp(g), 1, 8, p, None, None) == nv.VIT_ERR_ALIGN
+    n = ctypes.c_int(-1)
+    assert lib.vit_op_window_attention(p, 64, p, 0, p, None, None) == nv.VIT_ERR_ARG       # no windows
+    assert lib.vit_op_window_attention(p, 64, p, 17, p, None, None) == nv.VIT_ERR_ARG      # > P / 4
+    assert lib.vit_op_window_attention(p, 64, None, 1, p, None, None) == nv.VIT_ERR_ARG
+    assert lib.vit_op_window_attention(ctypes.c_void_p(0x10002), 64, p, 1, p, None, None) == nv.VIT_ERR_ALIGN
+    assert lib.vit_op_window_attention(p, (1 << 21) + 4, p, 1, p, None, None) == nv.VIT_ERR_LIMIT
+    assert lib.vit_op_window_positions(nv._gp(g), 1, 0, 5, p, p, p, p, ctypes.byref(n), None) == nv.VIT_ERR_ARG
+    assert lib.vit_op_window_positions(nv._gp(g), 1, 2, 8, p, p, p, p, ctypes.byref(n), None) == nv.VIT_ERR_ARG
+    assert lib.vit_op_window_positions(nv._gp(g), 1, 0, 8, p, p, p, p, None, None) == nv.VIT_ERR_ARG
     bad = np.array([[1, 7, 8]], np.int32)
-    assert lib.vit_op_window_attention(p, nv._gp(bad), 1, 8, p, None, None) == nv.VIT_ERR_GRID
-    assert lib.vit_op_window_positions(nv._gp(g), 1, 0, 5, p, p, p, None) == nv.VIT_ERR_ARG
-    assert lib.vit_op_window_positions(nv._gp(g), 1, 2, 8, p, p, p, None) == nv.VIT_ERR_ARG
+    assert lib.vit_op_window_positions(nv._gp(bad), 1, 0, 8, p, p, p, p, ctypes.byref(n), None) == nv.VIT_ERR_GRID
+    assert n.value == -1                                   # nothing written on an error
     assert lib.vit_op_gather_rows(p, p, p, 4, 2352 + 8, None) == nv.VIT_ERR_ALIGN
 
 
@@ -105,3 +110,20 @@ def test_mrope_rejects_bad_arguments(lib):
     assert lib.mrope_index(ctypes.c_void_p(16), 5, nv._gp(g), 1, ctypes.c_void_p(16), None, None, None) == nv.VIT_ERR_GRID
     assert lib.mrope_index(ctypes.c_void_p(16), 5, None, 1, ctypes.c_void_p(16), None, None, None) == nv.VIT_ERR_ARG
     assert lib.mrope_index(ctypes.c_void_p(16), -1, None, 0, ctypes.c_void_p(16), None, None, None) == nv.VIT_ERR_ARG
+
+
+def test_decoder_steps_reject_bad_arguments_before_cuda(lib):
+    from resolution_vit_vision_b200 import native as nv
+    p = ctypes.c_void_p(0x10000)
+    sec = np.array([16, 24, 24], np.int32)
+    bad_sec = np.array([16, 24, 23], np.int32)
+    ok = sec.ctypes.data_as(nv.c_i32p)
+    assert lib.mrope_apply(p, 28, p, 4, 128, p, 10, 1e6, bad_sec.ctypes.data_as(nv.c_i32p), None) == nv.VIT_ERR_ARG
+    assert lib.mrope_apply(p, 28, p, 4, 120, p, 10, 1e6, ok, None) == nv.VIT_ERR_ARG           # not a multiple of 16
+    assert lib.mrope_apply(None, 28, p, 4, 128, p, 10, 1e6, ok, None) == nv.VIT_ERR_ARG        # q missing
+    assert lib.mrope_apply(p, 28, p, 4, 128, None, 10, 1e6, ok, None) == nv.VIT_ERR_ARG        # positions missing
+    assert lib.mrope_apply(ctypes.c_void_p(0x10008), 28, p, 4, 128, p, 10, 1e6, ok, None) == nv.VIT_ERR_ALIGN
+    assert lib.scatter_vision_tokens(p, 10, p, 100, 12, p, 2, p, None, None) == nv.VIT_ERR_ARG  # dim % 8
+    assert lib.scatter_vision_tokens(p, (1 << 18) + 1, p, 100, 64, p, 2, p, None, None) == nv.VIT_ERR_ARG
+    assert lib.scatter_vision_tokens(p, 10, p, 100, 64, None, 2, p, None, None) == nv.VIT_ERR_ARG
+    assert lib.scatter_vision_tokens(p, 10, ctypes.c_void_p(0x10004), 100, 64, p, 2, p, None, None) == nv.VIT_ERR_ALIGN

@@ -32,9 +32,11 @@ def _window_cu(grids, order, window):
 @pytest.mark.parametrize("window", [8, 4, 16])
 def test_window_positions(order, window):
     grids = RAGGED
-    pos, mr, src = (to_np(t).astype(np.int64) for t in nv.op_window_positions(grids, order, window))
+    pos, mr, src, tab = (to_np(t).astype(np.int64) for t in nv.op_window_positions(grids, order, window))
     groups = vo.window_groups(grids, order, window)
     cu = _window_cu(grids, order, window)
+    np.testing.assert_array_equal(tab[:, 0], cu[:-1])      # the window table: first row, rows
+    np.testing.assert_array_equal(tab[:, 1], np.diff(cu))
     for i, g in enumerate(groups):      # window i is the contiguous run cu[i] .. cu[i + 1]
         assert sorted(src[cu[i]:cu[i + 1]].tolist()) == g.tolist()
     if order == 0:
@@ -77,7 +79,8 @@ def test_window_attention_kernel(grids, window):
     qkv = syn.make_matrix((P, 3840), 73 + P, 1.0)
     out = torch.full((P, 1280), float("nan"), dtype=torch.bfloat16, device=DEV)
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
-    nv.op_window_attention(bf16_bits_to_torch(qkv), grids, window, out, status=st)
+    tab = nv.op_window_positions(grids, 0, window)[3]
+    nv.op_window_attention(bf16_bits_to_torch(qkv), tab, out, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     x = vo._f64(qkv)
@@ -97,7 +100,8 @@ def test_window_attention_kernel_full_mixed_batch_peaked():
     qkv = syn.make_matrix((P, 3840), 74, 4.0)
     out = torch.empty((P, 1280), dtype=torch.bfloat16, device=DEV)
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
-    nv.op_window_attention(bf16_bits_to_torch(qkv), grids, 8, out, status=st)
+    tab = nv.op_window_positions(grids, 0, 8)[3]
+    nv.op_window_attention(bf16_bits_to_torch(qkv), tab, out, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     x = vo._f64(qkv)
