@@ -379,20 +379,38 @@ def main():
     ms = vd.max_over_ranks(ms, device=dev)
     assert enc.device_status() == 0
 
-    # ---- e2e: host (pinned) patches in, host tokens out, through vit_encode_host
+    # ---- e2e: host (pinned) patches in, host tokens out, through vit_encode_host. Two handles on
+    # two streams take alternate steps, so one step's copies overlap the other's kernels (the way a
+    # caller streams batches through the public API). Every step still copies its whole input in
+    # and its whole output back; the per-step working set (1.35 GB of weights read per encode)
+    # is far larger than L2, so no flush is needed between steps here.
     hp = patches.cpu().pin_memory()
-    ho = torch.empty((M4, wl.out_dim), dtype=torch.bfloat16).pin_memory()
-    for _ in range(2):
-        enc.encode_host(hp, wl.grids, ho)
+    ho = [torch.empty((M4, wl.out_dim), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    enc2 = nv.VisionEncoder(wts, wl.out_dim, window=args.window, full_blocks=full_blocks)
+    enc2.reserve(P)
+    encs = [enc, enc2]
+    streams = [stream, torch.cuda.Stream(device=dev)]
+    for e in encs:
+        if not args.no_graph:
+            e.graph_enable(True)
+    for i in range(4):
+        encs[i % 2].encode_host(hp, wl.grids, ho[i % 2], stream=streams[i % 2])
     torch.cuda.synchronize()
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(streams[0])
+    streams[1].wait_event(e_start)
     for i in range(args.steps):
-        flush.zero_()
-        ev2[i][0].record(stream)
-        enc.encode_host(hp, wl.grids, ho)
-        ev2[i][1].record(stream)
+        encs[i % 2].encode_host(hp, wl.grids, ho[i % 2], stream=streams[i % 2])
+    streams[0].wait_stream(streams[1])
+    e_end.record(streams[0])
     torch.cuda.synchronize()
-    e2e_ms = vd.max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev2])), device=dev)
+    if world > 1:
+        dist.barrier()
+    e2e_ms = vd.max_over_ranks(e_start.elapsed_time(e_end) / args.steps, device=dev)
+    assert enc2.device_status() == 0
+    enc2.close()
 
     pk, pk_kind = peaks()
     tc_peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
@@ -445,7 +463,10 @@ def main():
                 "tflops": achieved_total,
                 "e2e": {"value": units / (e2e_ms * 1e-3), "unit": "patches/s",
                         "h2d_bytes_per_step": P * syn.PATCH_K * 2, "d2h_bytes_per_step": M4 * wl.out_dim * 2,
-                        "ms_per_step": e2e_ms},
+                        "ms_per_step": e2e_ms,
+                        "how": "vit_encode_host, two handles on two streams taking alternate steps "
+                               "(copies of one step overlap the other's kernels); no L2 flush (the "
+                               "per-step working set of weights is far larger than L2)"},
                 "gpu_launches": int(launches),
                 "ms_per_step_profiled": ms_prof,
                 "roofline": roof,

@@ -150,7 +150,9 @@ int vit_graph_enable(vit_handle *h, int enable);
 
 /* vit_encode with HOST patches and HOST out (pinned memory gives asynchronous copies): copies
  * the patches into the handle's workspace, encodes, copies the tokens back, all on `stream`.
- * The host buffers must stay valid until the stream reaches that point. */
+ * The host buffers must stay valid until the stream reaches that point. With vit_graph_enable on,
+ * the encode between the two copies is replayed from a recorded graph as in vit_encode. To overlap
+ * one batch's copies with another's kernels, use one handle per stream (handles share weights). */
 int vit_encode_host(const void *host_patches, const int32_t *grid_thw, int n_images,
                     vit_handle *h, void *host_out, void *stream);
 

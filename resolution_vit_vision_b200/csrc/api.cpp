@@ -541,7 +541,8 @@ int vit_encode_host(const void *host_patches, const int32_t *grid_thw, int n_ima
     const size_t out_bytes = static_cast<size_t>(P / 4) * h->desc.out_dim * 2;
     if (cudaMemcpyAsync(h->patch_stage, host_patches, in_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return VIT_ERR_CUDA;
-    rc = encode_device(h, h->patch_stage, grid_thw, n_images, P, h->out_stage, s);
+    rc = (h->graph_on && !h->prof) ? encode_graph(h, h->patch_stage, grid_thw, n_images, P, h->out_stage, s)
+                                   : encode_device(h, h->patch_stage, grid_thw, n_images, P, h->out_stage, s);
     if (rc != VIT_OK) return rc;
     if (cudaMemcpyAsync(host_out, h->out_stage, out_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return VIT_ERR_CUDA;

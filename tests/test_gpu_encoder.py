@@ -171,6 +171,13 @@ def test_graph_replay_matches_direct_launches():
     torch.cuda.synchronize()
     np.testing.assert_array_equal(to_np(out), ref)
     assert (enc.launch_count() - n0) % 2 == 0 and enc.launch_count() > n0
+    # host buffers through the replayed graph
+    hp = p1.cpu().pin_memory()
+    ho = torch.empty((ref.shape[0], 1536), dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        enc.encode_host(hp, grids, ho)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(ho.float().numpy(), ref)
     # new data in the same buffers is encoded by the replay
     p2 = bf16_bits_to_torch(syn.make_patches(grids, 15))
     p1.copy_(p2)
