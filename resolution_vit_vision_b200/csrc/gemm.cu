@@ -4,10 +4,17 @@
 // table: Patchify 14x14 as a [P,1176]x[1176,1280] product, the ViT blocks' QKV / out-proj /
 // MLP linears, and the Patch Merger's two linears).
 //
-// Per CTA (one per SM, persistent over output tiles of 128 x BN):
-//   warp 0      TMA producer: A and B tiles (128B-swizzled, K-major) into a STAGES-deep ring
-//   warp 1      MMA issuer (one thread): tcgen05.mma 128xBNx16 into a TMEM accumulator;
-//               two accumulators so the epilogue of tile i overlaps the mainloop of tile i+1
+// Two SMs share each output tile of 256 x BN (a cluster of two CTAs, tcgen05 cta_group::2): each
+// CTA holds its 128 rows of A and half of the tile's BN rows of B in its own shared memory, so
+// every SM streams 64 bytes of operands per 128 x BN x 16 product share instead of 96 -- the
+// operand feed from L2, not the tensor pipe, had bounded the one-SM tiles. The even CTA issues
+// the M = 256 products; each CTA receives its 128 rows of the accumulator in its own TMEM.
+// Per CTA (persistent, the pair walks the 256 x BN tiles together):
+//   warp 0      TMA producer: its A rows and its half of B (128B-swizzled, K-major) into a
+//               STAGES-deep ring; both CTAs' loads complete on the even CTA's barrier
+//   warp 1      (even CTA, one thread) MMA issuer: tcgen05.mma 256xBNx16 into the pair's TMEM
+//               accumulators, commits multicast to both CTAs; two accumulators so the epilogue of
+//               tile i overlaps the mainloop of tile i+1
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (one row per thread), bias,
 //               GELU / 2-D rope, then the tile leaves through a double-buffered swizzled shared
 //               staging chunk and a TMA store -- or a TMA reduce-add into the fp32 residual
@@ -26,9 +33,9 @@ constexpr int kEpiBarrier = 1;    // named barrier of the 128 epilogue threads
 
 template <int BN>
 struct GemmShape {
-    static constexpr int STAGES = 4;
+    static constexpr int STAGES = BN == 240 ? 5 : 6;
     static constexpr int A_BYTES = kBM * kBK * 2;
-    static constexpr int B_BYTES = BN * kBK * 2;
+    static constexpr int B_BYTES = (BN / 2) * kBK * 2;   // this CTA's half of the B tile
     static constexpr int ACC_STRIDE = 256;    // TMEM columns between the two accumulators
     static constexpr int TMEM_COLS = 512;
     // output staging chunk: 128 rows x 128 bytes (32 fp32 or 64 bf16 columns), or for QKV one
@@ -45,7 +52,7 @@ struct GemmParams {
     const float2 *rope_cs;
     int32_t *status;
     int M, N, K;
-    int m_tiles, n_tiles, k_blocks;
+    int m_tiles, n_tiles, k_blocks;   // m_tiles: 256-row tiles of the CTA pair
 };
 
 // GELU(x) = x Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), with erf from Abramowitz & Stegun,
@@ -125,24 +132,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();                 // 0: issues the pair's products
+    const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S::STAGES; ++s) {
-            mbar_init(full + s, 1);
-            mbar_init(empty + s, 1);
+            mbar_init(full + s, 1);                       // (used in CTA 0: both CTAs' loads land on it)
+            mbar_init(empty + s, 1);                      // the pair's products are done with stage s
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull + a, 1);
-            mbar_init(tempty + a, 128);
+            mbar_init(tempty + a, 8);                     // (CTA 0) the 4 + 4 epilogue warps of the pair
         }
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, S::TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();                                       // both CTAs' barriers exist before any remote use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const WaitCtx wc{abort_flag, p.status};
@@ -154,25 +164,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_prefetch(&tmb);
             int stage = 0;
             uint32_t phase = 0;
-            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-                const int m0 = (tile / p.n_tiles) * kBM, n0 = (tile % p.n_tiles) * BN;
+            for (int tile = cluster; tile < total; tile += n_clusters) {
+                // this CTA's 128 rows of the pair's 256, and its half of the BN rows of B
+                const int m0 = (tile / p.n_tiles) * 2 * kBM + static_cast<int>(rank) * kBM;
+                const int n0 = (tile % p.n_tiles) * BN + static_cast<int>(rank) * (BN / 2);
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!mbar_wait(empty + stage, phase ^ 1u, wc)) goto producer_done;
-                    mbar_expect_tx(full + stage, S::A_BYTES + S::B_BYTES);
-                    tma_load_2d(sA + stage * S::A_BYTES, &tma, full + stage, kb * kBK, m0);
-                    tma_load_2d(sB + stage * S::B_BYTES, &tmb, full + stage, kb * kBK, n0);
+                    const uint32_t bar0 = cluster_addr(full + stage, 0);
+                    if (rank == 0) mbar_expect_tx(full + stage, 2 * (S::A_BYTES + S::B_BYTES));
+                    tma_load_2d_pair(sA + stage * S::A_BYTES, &tma, bar0, kb * kBK, m0);
+                    tma_load_2d_pair(sB + stage * S::B_BYTES, &tmb, bar0, kb * kBK, n0);
                     if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
         producer_done:;
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(kBM, BN, false, false);
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_bf16(2 * kBM, BN, false, false);
             int stage = 0;
             uint32_t phase = 0;
             int local = 0;
-            for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+            for (int tile = cluster; tile < total; tile += n_clusters, ++local) {
                 const int acc = local & 1;
                 const uint32_t acc_phase = (local >> 1) & 1;
                 if (!mbar_wait(tempty + acc, acc_phase ^ 1u, wc)) break;
@@ -189,13 +202,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         // +32 bytes per 16-element K step inside the 128-byte swizzle atom
                         const uint64_t da = smem_desc(a_addr + k * 32, 16, 1024, kSwizzle128B);
                         const uint64_t db = smem_desc(b_addr + k * 32, 16, 1024, kSwizzle128B);
-                        mma_bf16_ss(d_tmem, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+                        mma_bf16_ss_pair(d_tmem, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
                     }
-                    mma_commit(empty + stage);
+                    mma_commit_pair(empty + stage, 0x3);
                     if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                mma_commit(tfull + acc);
+                mma_commit_pair(tfull + acc, 0x3);
             }
         }
     } else {
@@ -213,13 +226,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             fence_proxy_async_smem();
             named_bar_sync(kEpiBarrier, 128);
         };
+        const uint32_t tempty0 = cluster_addr(tempty, 0);   // CTA 0's accumulator-free barriers
+        // this warp's share of the accumulator is read: one arrival per warp on CTA 0's barrier
+        auto release_acc = [&](int acc) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty0 + acc * 8);
+        };
         int local = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+        for (int tile = cluster; tile < total; tile += n_clusters, ++local) {
             const int acc = local & 1;
             const uint32_t acc_phase = (local >> 1) & 1;
             if (!mbar_wait(tfull + acc, acc_phase, wc)) break;
             tc_fence_after();
-            const int m0 = (tile / p.n_tiles) * kBM, n0 = (tile % p.n_tiles) * BN;
+            const int m0 = (tile / p.n_tiles) * 2 * kBM + static_cast<int>(rank) * kBM, n0 = (tile % p.n_tiles) * BN;
             const uint32_t t0 = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * S::ACC_STRIDE;
             if (EPI == VIT_EPI_QKV_ROPE) {
 #pragma unroll 1
@@ -230,10 +250,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 5; ++c) reg_fence16(u + c * 16);
-                    if (hh == BN / 80 - 1) {   // accumulator fully read: hand it back to the MMA warp
-                        tc_fence_before();
-                        mbar_arrive(tempty + acc);
-                    }
+                    if (hh == BN / 80 - 1) release_acc(acc);   // accumulator fully read: hand it back
                     float v[80];
 #pragma unroll
                     for (int j = 0; j < 80; ++j) v[j] = __uint_as_float(u[j]);
@@ -270,10 +287,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_ld32(t0 + c * 32, u);
                     tmem_wait_ld();
                     reg_fence32(u);
-                    if (c == BN / 32 - 1) {
-                        tc_fence_before();
-                        mbar_arrive(tempty + acc);
-                    }
+                    if (c == BN / 32 - 1) release_acc(acc);
                     const int col0 = n0 + c * 32;
                     if (col0 < p.N) {                   // uniform across the CTA
                         float v[32];
@@ -302,10 +316,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_wait_ld();
                     reg_fence32(u);
                     reg_fence32(u + 32);
-                    if (c == BN / 64 - 1) {
-                        tc_fence_before();
-                        mbar_arrive(tempty + acc);
-                    }
+                    if (c == BN / 64 - 1) release_acc(acc);
                     const int col0 = n0 + c * 64;
                     if (col0 < p.N) {
                         float v[64];
@@ -337,9 +348,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (*abort_flag) __nanosleep(200000);   // let copies already in flight land before exit
+    cluster_sync();                          // no remote arrival or product still targets either CTA
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, S::TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
     }
 }
 
@@ -353,8 +365,8 @@ int gemm_make_a_map(CUtensorMap *map, const void *A, int64_t M, int K) {
 }
 
 int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue) {
-    const uint32_t bn = (epilogue == VIT_EPI_QKV_ROPE) ? 240 : 256;
-    return tmap_2d(map, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, N, static_cast<uint64_t>(K) * 2, vitk::kBK, bn,
+    const uint32_t bn = (epilogue == VIT_EPI_QKV_ROPE) ? 240 : 256;   // each CTA of a pair loads half
+    return tmap_2d(map, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, N, static_cast<uint64_t>(K) * 2, vitk::kBK, bn / 2,
                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -386,10 +398,31 @@ static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtens
             return VIT_ERR_CUDA;
         if (dev < 64) configured[dev] = true;
     }
+    static int max_clusters[64] = {};   // pairs that fit on the device at once (set with the attribute)
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(vitk::kGemmThreads);
+    cfg.dynamicSmemBytes = S::SMEM;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (dev < 64 && max_clusters[dev] == 0) {
+        cfg.gridDim = dim3(2 * 74);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, vitk::gemm_tc_kernel<BN, EPI>, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = device_sm_count() / 2;
+        }
+        max_clusters[dev] = n;
+    }
     const int total = p.m_tiles * p.n_tiles;
-    const int sms = device_sm_count();
-    const int grid = total < sms ? total : sms;
-    vitk::gemm_tc_kernel<BN, EPI><<<grid, vitk::kGemmThreads, S::SMEM, s>>>(ta, tb, tc, p);
+    const int pairs = dev < 64 ? max_clusters[dev] : device_sm_count() / 2;
+    cfg.gridDim = dim3(2 * (total < pairs ? total : pairs));
+    if (cudaLaunchKernelEx(&cfg, vitk::gemm_tc_kernel<BN, EPI>, ta, tb, tc, p) != cudaSuccess) return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 
@@ -405,7 +438,7 @@ int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap 
     p.M = static_cast<int>(M);
     p.N = N;
     p.K = K;
-    p.m_tiles = static_cast<int>((M + vitk::kBM - 1) / vitk::kBM);
+    p.m_tiles = static_cast<int>((M + 2 * vitk::kBM - 1) / (2 * vitk::kBM));
     p.k_blocks = (K + vitk::kBK - 1) / vitk::kBK;
     switch (epilogue) {
         case VIT_EPI_QKV_ROPE:
