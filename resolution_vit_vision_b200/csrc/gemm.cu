@@ -110,16 +110,24 @@ __device__ __forceinline__ void stage_row128(uint8_t *stg, int r, const uint32_t
 }
 
 // The 2-D rope on one 80-wide q or k head held in registers: pair (d, d+40) turns by the angle
-// of dim d, row position h for d < 20, column w for d >= 20.
+// of dim d, row position h for d < 20, column w for d >= 20. Two dims at a time (d and d + 1 lie on
+// the same side of 20) in packed fp32x2, like the GELU above.
 __device__ __forceinline__ void rope_head(float *v, int hw, const float2 *cs) {
     const float2 *ch = cs + (hw >> 16) * 20;
     const float2 *cw = cs + (hw & 0xFFFF) * 20;
 #pragma unroll
-    for (int d = 0; d < 40; ++d) {
-        const float2 c = __ldg(d < 20 ? ch + d : cw + (d - 20));
-        const float x0 = v[d], x1 = v[d + 40];
-        v[d] = x0 * c.x - x1 * c.y;
-        v[d + 40] = x1 * c.x + x0 * c.y;
+    for (int d = 0; d < 40; d += 2) {
+        const float2 a = __ldg(d < 20 ? ch + d : cw + (d - 20));       // (cos, sin) of dim d
+        const float2 b = __ldg(d < 20 ? ch + d + 1 : cw + (d - 19));   // and of dim d + 1
+        float t0, t1, u0, u1;
+        fmul2(t0, t1, v[d], v[d + 1], a.x, b.x);              // x0 cos
+        fmul2(u0, u1, v[d + 40], v[d + 41], a.x, b.x);        // x1 cos
+        ffma2(u0, u1, v[d], v[d + 1], a.y, b.y, u0, u1);      // x1 cos + x0 sin
+        ffma2(t0, t1, v[d + 40], v[d + 41], -a.y, -b.y, t0, t1);   // x0 cos - x1 sin
+        v[d] = t0;
+        v[d + 1] = t1;
+        v[d + 40] = u0;
+        v[d + 41] = u1;
     }
 }
 
