@@ -5,14 +5,22 @@
 // (image, frame); every query attends to every key of its own segment and to nothing else:
 // out = softmax(q k^T / sqrt(80)) v per segment and head (16 heads x 80).
 //
-// One CTA = one 128-query tile of one (segment, head). Keys stream through in tiles of 128:
-//   warp 0      TMA producer: Q once, K_j and V_j into a 3-deep ring (32-byte swizzle, the
-//               80-wide head read as five 16-column boxes straight from the [P, 3840] QKV buffer)
-//   warp 1      MMA issuer: S_j = Q K_j^T into one of two TMEM score buffers (M=128, N=128,
-//               K=5x16), then O += P_j V_j (M=128, N=80, K=8x16) into a TMEM output accumulator
-//   warps 2..5  softmax, one query row per thread: scores from TMEM, online max / sum in fp32,
-//               P in bf16 to shared memory (128B-swizzled, K-major), O rescaled in TMEM when the
-//               running max grows, final O / l written as bf16.
+// One CTA = two 128-query tiles (A and B) of one (segment, head); keys stream through in tiles
+// of 112 that both query tiles share:
+//   warp 0      TMA producer: Q of both tiles once, K_j and V_j into a 4-deep ring (32-byte
+//               swizzle, the 80-wide head read as five 16-column boxes straight from the [P, 3840]
+//               QKV buffer)
+//   warps 1, 2  one MMA-issuing thread per query tile: S_x(j) = Q_x K_j^T into the tile's TMEM
+//               score buffer (M=128, N=112, K=5x16), then O_x += P_x(j) V_j (M=128, N=80,
+//               K=7x16) with P_x read from TMEM
+//   warps 3..6  softmax of tile A, 7..10 of tile B, one query row per thread: scores from TMEM,
+//               online max / sum in fp32 with a lazy rescale (the exponent offset moves only when
+//               the running max, in log2 units, grows by more than 8), P in bf16 back to TMEM, O
+//               rescaled after the exponentials; the two warpgroups take turns at the
+//               exponentials (named barriers) so one group's loads and stores overlap the
+//               other's MUFU work; final O / l written as bf16.
+// Work items are (segment, pair of query tiles), longest segments first; the work list travels
+// as a kernel parameter.
 #include <cuda_bf16.h>
 
 #include <algorithm>
