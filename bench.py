@@ -322,7 +322,8 @@ def main():
         wl = dataclasses.replace(wl, depth=args.depth)
     P_job = sum(t * h * w for t, h, w in wl.grids)          # patches of one whole batch
     if args.shard and world > 1:                              # this rank's images of the one batch
-        _, my_grids, _ = vd.shard(wl.grids, rank, world, wl.depth)
+        fb = tuple(int(x) for x in args.full_blocks.split(",") if x) if args.window else ()
+        _, my_grids, _ = vd.shard(wl.grids, rank, world, wl.depth, args.window, fb)
         wl = dataclasses.replace(wl, grids=tuple(my_grids))
     full_blocks = tuple(int(x) for x in args.full_blocks.split(",") if x) if args.window else ()
     P, M4, flops_launch, ln_bytes, flops_total = work_model(wl.grids, wl.depth, wl.out_dim, args.window,
