@@ -46,8 +46,9 @@ def parse():
                     help="the windowed (Qwen2.5-VL) tower: window side in patches (8 = 112 px); 0 = Qwen2-VL")
     ap.add_argument("--full-blocks", default="7,15,23,31",
                     help="with --window: the full-attention blocks (0-based, comma-separated)")
-    ap.add_argument("--op", default=None, choices=["mrope_apply", "scatter"],
-                    help="time one decoder-side step on the prompt that carries the workload's merged tokens")
+    ap.add_argument("--op", default=None, choices=["mrope_apply", "scatter", "mrope_index", "yardstick"],
+                    help="time one decoder-side step on the prompt that carries the workload's merged "
+                         "tokens, or (yardstick) library GEMM / attention on the encoder's shapes")
     return ap.parse_args()
 
 
@@ -198,7 +199,11 @@ def cpu_baseline(wl, budget_s=25.0, window=0, full_blocks=()):
         if el * (done + 1) / done > budget_s:
             break
     el = time.perf_counter() - t0
-    return {"value": done * P / el, "unit": "patches/s", "cores": int(cores), "kind": "oracle",
+    try:
+        cpu = next(l.split(":", 1)[1].strip() for l in open("/proc/cpuinfo") if l.startswith("model name"))
+    except (OSError, StopIteration):
+        cpu = "unknown"
+    return {"value": done * P / el, "unit": "patches/s", "cores": int(cores), "kind": "oracle", "cpu": cpu,
             "sample": f"image {i} of the batch (grid {tuple(g[0])}, {P} patches) through the full "
                       f"depth-{wl.depth} fp64 oracle{' (windowed)' if window else ''}, {done} pass(es), "
                       f"{el:.1f} s"}
@@ -251,7 +256,14 @@ def run_op(args):
     t_ids = torch.from_numpy(ids.astype(np.int32)).to(dev)
     g = torch.Generator(device=dev)
     g.manual_seed(wl.seed)
-    if args.op == "mrope_apply":
+    if args.op == "mrope_index":   # latency-bound: one CTA walks the prompt
+        pos = torch.empty((3, L), dtype=torch.int32, device=dev)
+        delta = torch.empty((1,), dtype=torch.int32, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        step = lambda: nv.mrope_index(t_ids, grids, out=pos, delta=delta, status=st)
+        nbytes = 4 * L + 12 * L
+        unit_desc = "ids read (4 L bytes), [3, L] int32 ids written (12 L bytes)"
+    elif args.op == "mrope_apply":
         pos, _ = nv.mrope_index(t_ids, grids)
         q = torch.randn((L, 28, 128), generator=g, device=dev).to(torch.bfloat16)
         k = torch.randn((L, 4, 128), generator=g, device=dev).to(torch.bfloat16)
@@ -279,7 +291,7 @@ def run_op(args):
         step()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
-    if args.op == "scatter":
+    if args.op in ("scatter", "mrope_index"):
         assert int(st.item()) == 0
     ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
     pk, pk_kind = peaks()
@@ -293,11 +305,65 @@ def run_op(args):
     return 0
 
 
+# ------------------------------------------------------------------------------ library yardstick
+def run_yardstick(args):
+    """Context, not the product: the same contractions through libraries (torch's cuBLAS linear for
+    the four layer GEMM shapes, torch scaled_dot_product_attention per segment for the block-diagonal
+    attention), timed like the encoder's kernels (CUDA events, L2 flushed before each call)."""
+    import torch
+    import torch.nn.functional as F
+    from resolution_vit_vision_b200 import synthetic as syn
+    wl = syn.WORKLOADS[args.workload]
+    P = sum(t * h * w for t, h, w in wl.grids)
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def timed(fn, reps=10):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    out = {"op": "yardstick", "config": {"workload": f"{wl.name}: {wl.description}", "patches": P},
+           "gemm": {}, "attention": {}}
+    for name, N, K in [("qkv", 3840, 1280), ("out_proj", 1280, 1280), ("fc1", 5120, 1280), ("fc2", 1280, 5120)]:
+        A = torch.randn((P, K), device=dev).to(torch.bfloat16)
+        W = (torch.randn((N, K), device=dev) * 0.02).to(torch.bfloat16)
+        bias = torch.zeros(N, device=dev, dtype=torch.bfloat16)
+        ms = timed(lambda: F.linear(A, W, bias))
+        out["gemm"][name] = {"library": "torch F.linear (cuBLAS)", "ms": ms, "tflops": 2.0 * P * N * K / (ms * 1e-3) / 1e12}
+    qkv = torch.randn((P, 3, 16, 80), device=dev).to(torch.bfloat16)
+    segs = [h * w for t, h, w in wl.grids for _ in range(t)]
+    starts = np.concatenate([[0], np.cumsum(segs)])
+
+    def attn():
+        for i, n in enumerate(segs):
+            x = qkv[starts[i]:starts[i] + n]
+            q, k, v = (x[:, j].transpose(0, 1).unsqueeze(0) for j in range(3))
+            F.scaled_dot_product_attention(q, k, v)
+    ms = timed(attn)
+    flops = 4.0 * 1280 * sum(n * n for n in segs)
+    out["attention"] = {"library": "torch scaled_dot_product_attention, one call per segment", "ms": ms,
+                        "tflops": flops / (ms * 1e-3) / 1e12}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------------------ native arm
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "yardstick":
+        return run_yardstick(args)
     if args.op:
         return run_op(args)
     import torch
