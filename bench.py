@@ -8,6 +8,14 @@ out 3584). N > 1 (launched with torch.distributed.run): every rank encodes its o
 scaling, no collective on the data path); time = max over ranks of the CUDA-event step time.
 Rank 0 prints one JSON line. ``--impl reference`` times the CPU oracle on a bounded sample of
 the same workload instead (rank 0 only).
+
+The line also carries ``e2e`` (the same metric through vit_encode_host with pinned host buffers,
+copies inside the timed region; two handles on two streams take alternate steps), the per-kernel
+split of a second pass with events around every launch, the roofline of the dominant kernel, the
+SM clocks sampled during the timed region and the CPU baseline. Other modes: ``--window 8`` (the
+windowed tower), ``--shard`` (N > 1: one batch split by image), ``--op mrope_apply|scatter|
+mrope_index`` (decoder-side steps), ``--op yardstick`` (library GEMM / attention on the same
+shapes, for context).
 """
 from __future__ import annotations
 
