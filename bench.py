@@ -243,7 +243,7 @@ def run_reference(args):
                        "full_blocks": list(full_blocks)},
             "merged_tokens_per_s": v / 4,
             "cpu_baseline": {"value": v, "unit": "patches/s", "cores": vals[0]["cores"], "kind": "oracle",
-                             "sample": vals[0]["sample"]},
+                             "cpu": vals[0]["cpu"], "sample": vals[0]["sample"]},
             "e2e": {"value": v, "unit": "patches/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
