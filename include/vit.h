@@ -159,13 +159,17 @@ int vit_encode_host(const void *host_patches, const int32_t *grid_thw, int n_ima
 /* 3-D M-RoPE position ids for the decoder ("Qwen2-VL" intro and Qwen2VLModel table, mrope;
  * LiteRT-LM card, M-RoPE note). input_ids: int32 [L]. grid_thw: HOST int32 [n_grids, 3], the
  * grids of the prompt's images and videos in order of appearance (n_grids may be 0; unused
- * trailing grids are ignored). out: int32 [3, L] (t, h, w axes). delta: int32 [1] or NULL,
- * receives (largest id + 1) - L. dev_status: int32 [1] or NULL; on a malformed prompt the kernel
- * writes VIT_ERR_TOKENS there and leaves out/delta untouched (with NULL the error is silent).
+ * trailing grids are ignored, their values are not even checked). out: int32 [3, L] (t, h, w
+ * axes). delta: int32 [1] or NULL, receives (largest id + 1) - L. dev_status: int32 [1] or NULL;
+ * on a malformed prompt the kernel writes VIT_ERR_TOKENS there and leaves out/delta untouched
+ * (with NULL the error is silent). Malformed means: a vision run whose length is not the
+ * t*(h/2)*(w/2) of the grid it consumes, a vision run with no grid left, or a consumed grid with
+ * t < 1, h or w odd or < 2, or a run length above L.
  * The rule: text tokens (incl. vision_start/end) take (c, c, c) from a cursor c that counts up;
  * a vision run follows a vision_start, is t*(h/2)*(w/2) image or video tokens, its j-th token
  * takes c + (j / (h'w'), (j / w') % h', j % w'), then c += max(t, h', w').
- * Host-side returns: VIT_ERR_ARG (NULL pointers, L < 0, n_grids out of range), VIT_ERR_GRID. */
+ * Host-side returns: VIT_ERR_ARG (NULL pointers, L < 0, n_grids out of range), VIT_ERR_LIMIT
+ * (L > 2^30). */
 int mrope_index(const int32_t *input_ids, int64_t L, const int32_t *grid_thw, int n_grids,
                 int32_t *out, int32_t *delta, int32_t *dev_status, void *stream);
 
@@ -177,18 +181,26 @@ int mrope_index(const int32_t *input_ids, int64_t L, const int32_t *grid_thw, in
  * computes exactly what vit_encode computes, with the activations in a fixed file-scope device
  * array inside the library, and it calls no cudaMalloc, cudaFree or other allocating routine.
  *   - Limit: at most VIT_NOALLOC_MAX_PATCHES patches per call (the sum of t*h*w), so the array
- *     is about 26.3 MB (activations of 1024 patches + the rope table). Every GPU that loads the
- *     library holds it from load until process exit. Larger batches return VIT_ERR_LIMIT and
+ *     is about 26.3 MB (activations of 1024 patches + the rope table). Every GPU on which the
+ *     array has been set up holds it until process exit. Larger batches return VIT_ERR_LIMIT and
  *     launch nothing.
- *   - The first call on a device sets the array up on that device (looks up its device address
- *     and fills its rope table with one kernel on `stream`); make that first call before any
- *     stream capture.
+ *   - The first call on a device sets the array up on that device: it looks up the array's
+ *     device address and fills its rope table with one kernel on `stream`, then waits for that
+ *     kernel (a synchronize of `stream`), so later calls on any stream find the table ready.
+ *     Under CUDA's default lazy module loading, that first call is also when the library's
+ *     module holding the array is loaded on the device, i.e. when the array's 26.3 MB are
+ *     allocated. Make the first call on each device at start-up, before another allocator
+ *     takes the device's memory and before any stream capture (or run with
+ *     CUDA_MODULE_LOADING=EAGER, which allocates the array when the CUDA context is created).
+ *     Every later call allocates nothing and does not synchronise.
  *   - Every call, on every stream, shares the one array and leaves the last call's activations in
  *     it. Calls whose work overlaps on the GPU race with each other: issue them on one stream or
  *     order them. Nothing in the array needs clearing between calls: each buffer is fully
  *     written before it is read.
  *   - Arguments as for vit_encode; weights from vit_weights_create on the current device, made
- *     without windows (desc.window == 0; a windowed handle returns VIT_ERR_ARG).
+ *     without windows (desc.window == 0; a windowed handle returns VIT_ERR_ARG). A grid row with
+ *     h or w above VIT_NOALLOC_MAX_PATCHES / 2, or t above VIT_NOALLOC_MAX_PATCHES / 4, returns
+ *     VIT_ERR_LIMIT before any product of its values is formed.
  *     dev_status: int32 [1] device or NULL; a kernel wait that timed out writes VIT_ERR_TIMEOUT
  *     there (it is not cleared by the call). */
 #define VIT_NOALLOC_MAX_PATCHES 1024

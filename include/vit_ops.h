@@ -64,6 +64,15 @@ int vit_op_layernorm(const float *X, const void *gamma, const void *beta, void *
 int vit_op_attention(const void *qkv, int64_t P, const int32_t *cu_seqlens, int n_seg, void *out,
                      int32_t *dev_status, void *stream);
 
+/* The exponential that the attention softmax computes on the FMA pipe for a share of its scores
+ * (no counterpart on the pages, which fix only softmax itself: "Qwen2-VL-2B-Instruct --
+ * LiteRT-LM", Vision row, full attention). y[i] = 2^x[i] for x, y fp32 [n] device, n >= 0: range
+ * reduction x = j + f (j = rint x, |f| <= 1/2), 2^f by a degree-3 minimax polynomial, j added to
+ * the exponent; relative error <= 7.5e-5 for x in [-125, 127); 0 for x <= -127.5 (and -inf);
+ * between those, 0 or a value of at most 2^-124 (2^f's exponent field may underflow there). |x| must stay below 2^22 (inputs beyond are not
+ * rejected and give meaningless results). */
+int vit_op_exp2_fma(const float *x, float *y, int64_t n, void *stream);
+
 /* Window order of the windowed (Qwen2.5-VL) tower ("Qwen2.5-VL-7B-Instruct", inference-research
  * model record, architecture note: 112-px windows). Rows in window order run, per image and frame,
  * over the windows of window x window patches (window even, >= 2) in raster order, inside a window

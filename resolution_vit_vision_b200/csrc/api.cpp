@@ -555,11 +555,7 @@ int mrope_index(const int32_t *input_ids, int64_t L, const int32_t *grid_thw, in
     if (L > 0 && (!input_ids || !out)) return VIT_ERR_ARG;
     if (n_grids > 0 && !grid_thw) return VIT_ERR_ARG;
     if (L > (int64_t(1) << 30)) return VIT_ERR_LIMIT;
-    for (int i = 0; i < n_grids; ++i) {
-        const int t = grid_thw[3 * i], hh = grid_thw[3 * i + 1], ww = grid_thw[3 * i + 2];
-        if (t < 1 || hh < 2 || ww < 2 || (hh & 1) || (ww & 1)) return VIT_ERR_GRID;
-        if (static_cast<int64_t>(t) * (hh / 2) * (ww / 2) > (int64_t(1) << 30)) return VIT_ERR_LIMIT;
-    }
+    // grid values are checked on the device, only for the grids the prompt's vision runs consume
     return vith::mrope_launch(input_ids, L, grid_thw, n_grids, out, delta, dev_status,
                               static_cast<cudaStream_t>(stream));
 }
@@ -655,6 +651,11 @@ int vit_op_attention(const void *qkv, int64_t P, const int32_t *cu_seqlens, int 
     const int rc = vith::attn_make_maps(&t, qkv, P);
     if (rc != VIT_OK) return rc;
     return vith::attn_launch(t, cu_seqlens, n_seg, out, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+int vit_op_exp2_fma(const float *x, float *y, int64_t n, void *stream) {
+    if (n < 0 || (n > 0 && (!x || !y))) return VIT_ERR_ARG;
+    return vith::exp2_fma_launch(x, y, n, static_cast<cudaStream_t>(stream));
 }
 
 int vit_op_window_positions(const int32_t *grid_thw, int n_images, int patch_order, int window, int32_t *pos,

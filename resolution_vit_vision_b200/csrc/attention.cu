@@ -16,9 +16,11 @@
 //   warps 3..6  softmax of tile A, 7..10 of tile B, one query row per thread: scores from TMEM,
 //               online max / sum in fp32 with a lazy rescale (the exponent offset moves only when
 //               the running max, in log2 units, grows by more than 8), P in bf16 back to TMEM, O
-//               rescaled after the exponentials; the two warpgroups take turns at the
-//               exponentials (named barriers) so one group's loads and stores overlap the
-//               other's MUFU work; final O / l written as bf16.
+//               rescaled after the exponentials; the two warpgroups take turns at the MUFU
+//               (named barriers) so one group's loads and stores overlap the other's MUFU work,
+//               and a fixed share of every row's exponentials runs on the FMA pipe instead
+//               (exp2_fma2: range reduction + a minimax polynomial), computed before the
+//               group's MUFU turn, while the other group holds the MUFU; final O / l in bf16.
 // Work items are (segment, pair of query tiles), longest segments first; the work list travels
 // as a kernel parameter.
 #include <cuda_bf16.h>
@@ -46,6 +48,15 @@ constexpr int kMaxWorkPerLaunch = 4096;
 // Lazy rescaling: a row's exponent offset only moves when its running max grows by more than
 // this (log2 units), so P stays below 2^8 and O is rarely rescaled.
 constexpr float kRescaleThreshold = 8.0f;
+// Exponentials split between the two pipes: of every kFmaPeriod pairs of P columns, the first
+// kFmaPairs are computed on the FMA pipe (exp2_fma2), the others by the MUFU (ex2.approx). The
+// MUFU takes one warp instruction per 8 cycles on a sub-partition; one FMA-pipe exponential
+// costs about eight issue slots, so a small share balances the two.
+#ifndef VIT_ATTN_FMA_PAIRS
+#define VIT_ATTN_FMA_PAIRS 0
+#endif
+constexpr int kFmaPeriod = 8, kFmaPairs = VIT_ATTN_FMA_PAIRS;
+__host__ __device__ constexpr bool fma_pair(int i) { return (i % kFmaPeriod) < kFmaPairs; }
 // TMEM columns of query tile x: scores S_x (112), P_x (bf16 pairs, 56 used of 64), O_x (80).
 __host__ __device__ constexpr uint32_t col_s(int x) { return x * 112; }
 __host__ __device__ constexpr uint32_t col_p(int x) { return 224 + x * 64; }
@@ -253,18 +264,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float neg_m = -m_used;
             float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             uint32_t pk[56];
-            named_bar_sync(my_turn, 256);                           // this group's turn
-            // groups of four pairs: eight independent exponentials in flight before their results
-            // are summed and packed, so the MUFU latency overlaps within one thread
+            // the FMA-pipe share first, while the other group holds the MUFU
+#pragma unroll
+            for (int i = 0; i < kBKV / 2; ++i) {
+                if (!fma_pair(i)) continue;
+                float p0 = fmaf(__uint_as_float(sr[2 * i]), scale_log2, neg_m);
+                float p1 = fmaf(__uint_as_float(sr[2 * i + 1]), scale_log2, neg_m);
+                exp2_fma2(p0, p1);
+                r8[(i & 3) + 4 * ((i >> 2) & 1)] += p0 + p1;
+                pk[i] = pack_bf16x2(p0, p1);
+            }
+            named_bar_sync(my_turn, 256);                           // this group's MUFU turn
+            // groups of four pairs: up to eight independent exponentials in flight before their
+            // results are summed and packed, so the MUFU latency overlaps within one thread
 #pragma unroll
             for (int k = 0; k < kBKV; k += 8) {
                 float p[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) p[e] = fmaf(__uint_as_float(sr[k + e]), scale_log2, neg_m);
+                for (int e = 0; e < 8; ++e)
+                    if (!fma_pair((k + e) >> 1)) p[e] = fmaf(__uint_as_float(sr[k + e]), scale_log2, neg_m);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) p[e] = ex2(p[e]);
+                for (int e = 0; e < 8; ++e)
+                    if (!fma_pair((k + e) >> 1)) p[e] = ex2(p[e]);
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
+                    if (fma_pair((k + e) >> 1)) continue;
                     r8[(e >> 1) + 4 * ((k >> 3) & 1)] += p[e] + p[e + 1];
                     pk[(k + e) >> 1] = pack_bf16x2(p[e], p[e + 1]);
                 }
@@ -332,9 +356,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
 }
 
+// y[i] = exp2_fma2(x[i]): the FMA-pipe exponential of the softmax, elementwise, so that its error
+// can be checked on a dense sweep against the exact 2^x.
+__global__ void exp2_fma_kernel(const float *__restrict__ x, float *__restrict__ y, int64_t n) {
+    for (int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x); i < n;
+         i += 2 * static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float a = x[i], b = i + 1 < n ? x[i + 1] : 0.0f;
+        exp2_fma2(a, b);
+        y[i] = a;
+        if (i + 1 < n) y[i + 1] = b;
+    }
+}
+
 }  // namespace vitk
 
 namespace vith {
+
+int exp2_fma_launch(const float *x, float *y, int64_t n, cudaStream_t s) {
+    if (n <= 0) return VIT_OK;
+    const int64_t pairs = (n + 1) / 2;
+    const int blocks = static_cast<int>(std::min<int64_t>((pairs + 255) / 256, 148 * 16));
+    vitk::exp2_fma_kernel<<<blocks, 256, 0, s>>>(x, y, n);
+    return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
+}
+
 
 // Two views of the [P, 3840] QKV buffer, 16-column boxes with 32-byte swizzle: query tiles of
 // 128 rows and key / value tiles of kBKV rows.
@@ -347,51 +392,71 @@ int attn_make_maps(AttnMaps *m, const void *qkv, int64_t P) {
     return rc;
 }
 
-// cu_seqlens: HOST [n_seg + 1]. Builds the (segment, q-tile) list, longest segments first,
-// and launches as many kernels as the per-launch limits need.
-int attn_launch(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
-                cudaStream_t s) {
-    static bool configured[64] = {};
+namespace {
+
+bool configure_attention() {
+    static bool configured[64] = {};   // the attribute is set once per device
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !configured[dev]) {
-        if (cudaFuncSetAttribute(vitk::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, vitk::kAttnSmem) !=
-            cudaSuccess)
-            return VIT_ERR_CUDA;
-        configured[dev] = true;
+    if (dev < 64 && configured[dev]) return true;
+    if (cudaFuncSetAttribute(vitk::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, vitk::kAttnSmem) !=
+        cudaSuccess)
+        return false;
+    if (dev < 64) configured[dev] = true;
+    return true;
+}
+
+// Packs the (segment, pair of query tiles) work of the segments in `order` into as many launches
+// as the per-launch tables need. A segment whose tiles do not all fit into the current launch
+// continues in the next one (its start and length are repeated there), so one segment of any
+// length up to VIT_MAX_PATCHES runs.
+int launch_plans(vitk::AttnPlan &plan, const int *order, int n_seg,
+                 const int32_t *cu_seqlens, const AttnMaps &tqkv, void *out, int32_t *status, cudaStream_t s) {
+    constexpr int kRowsPerItem = vitk::kBQ * vitk::kQTilesPerCta;
+    plan.n_seg = 0;
+    plan.n_work = 0;
+    auto flush = [&]() {
+        if (plan.n_work > 0) {
+            vitk::attn_tc_kernel<<<plan.n_work * VIT_HEADS, vitk::kAttnThreads, vitk::kAttnSmem, s>>>(
+                tqkv.q, tqkv.kv, plan, static_cast<__nv_bfloat16 *>(out), status);
+            if (cudaGetLastError() != cudaSuccess) return false;
+        }
+        plan.n_seg = 0;
+        plan.n_work = 0;
+        return true;
+    };
+    for (int i = 0; i < n_seg; ++i) {
+        const int sg = order[i];
+        const int len = cu_seqlens[sg + 1] - cu_seqlens[sg];
+        const int tiles = (len + kRowsPerItem - 1) / kRowsPerItem;
+        for (int t = 0; t < tiles;) {
+            if (plan.n_seg == vitk::kMaxSegPerLaunch || plan.n_work == vitk::kMaxWorkPerLaunch)
+                if (!flush()) return VIT_ERR_CUDA;
+            const int ls = plan.n_seg++;
+            plan.start[ls] = cu_seqlens[sg];
+            plan.len[ls] = len;
+            for (; t < tiles && plan.n_work < vitk::kMaxWorkPerLaunch; ++t) plan.work[plan.n_work++] = (ls << 16) | t;
+        }
     }
-    // segment order: longest first (longest-processing-time-first over the CTA waves)
+    return flush() ? VIT_OK : VIT_ERR_CUDA;
+}
+
+}  // namespace
+
+// cu_seqlens: HOST [n_seg + 1]. Builds the (segment, q-tile) list, longest segments first
+// (longest-processing-time-first over the CTA waves), and launches as many kernels as the
+// per-launch limits need.
+int attn_launch(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
+                cudaStream_t s) {
+    if (n_seg < 0 || n_seg > VIT_MAX_SEGMENTS) return VIT_ERR_LIMIT;
+    if (!configure_attention()) return VIT_ERR_CUDA;
     std::vector<int> order(n_seg);
     for (int i = 0; i < n_seg; ++i) order[i] = i;
     std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
         return (cu_seqlens[a + 1] - cu_seqlens[a]) > (cu_seqlens[b + 1] - cu_seqlens[b]);
     });
     auto plan = std::make_unique<vitk::AttnPlan>();
-    size_t pos = 0;
-    while (pos < order.size()) {
-        plan->n_seg = 0;
-        plan->n_work = 0;
-        while (pos < order.size()) {
-            const int sg = order[pos];
-            const int len = cu_seqlens[sg + 1] - cu_seqlens[sg];
-            const int tiles = (len + vitk::kBQ * vitk::kQTilesPerCta - 1) / (vitk::kBQ * vitk::kQTilesPerCta);
-            if (plan->n_seg == vitk::kMaxSegPerLaunch || plan->n_work + tiles > vitk::kMaxWorkPerLaunch) {
-                if (plan->n_seg == 0) return VIT_ERR_LIMIT;   // one segment alone exceeds a launch
-                break;
-            }
-            const int ls = plan->n_seg++;
-            plan->start[ls] = cu_seqlens[sg];
-            plan->len[ls] = len;
-            for (int t = 0; t < tiles; ++t) plan->work[plan->n_work++] = (ls << 16) | t;
-            ++pos;
-        }
-        if (plan->n_work > 0) {
-            vitk::attn_tc_kernel<<<plan->n_work * VIT_HEADS, vitk::kAttnThreads, vitk::kAttnSmem, s>>>(
-                tqkv.q, tqkv.kv, *plan, static_cast<__nv_bfloat16 *>(out), status);
-            if (cudaGetLastError() != cudaSuccess) return VIT_ERR_CUDA;
-        }
-    }
-    return VIT_OK;
+    return launch_plans(*plan, order.data(), n_seg, cu_seqlens, tqkv, out, status, s);
 }
 
 // attn_launch with the schedule kept on the host stack and an in-place sort (ties broken by
@@ -399,15 +464,7 @@ int attn_launch(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg, void
 int attn_launch_stack(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
                       cudaStream_t s) {
     if (n_seg < 0 || n_seg > VIT_MAX_SEGMENTS) return VIT_ERR_LIMIT;
-    static bool configured[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !configured[dev]) {
-        if (cudaFuncSetAttribute(vitk::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, vitk::kAttnSmem) !=
-            cudaSuccess)
-            return VIT_ERR_CUDA;
-        if (dev < 64) configured[dev] = true;
-    }
+    if (!configure_attention()) return VIT_ERR_CUDA;
     int order[VIT_MAX_SEGMENTS];
     for (int i = 0; i < n_seg; ++i) order[i] = i;
     std::sort(order, order + n_seg, [&](int a, int b) {
@@ -415,31 +472,7 @@ int attn_launch_stack(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg
         return la != lb ? la > lb : a < b;
     });
     vitk::AttnPlan plan;
-    int pos = 0;
-    while (pos < n_seg) {
-        plan.n_seg = 0;
-        plan.n_work = 0;
-        while (pos < n_seg) {
-            const int sg = order[pos];
-            const int len = cu_seqlens[sg + 1] - cu_seqlens[sg];
-            const int tiles = (len + vitk::kBQ * vitk::kQTilesPerCta - 1) / (vitk::kBQ * vitk::kQTilesPerCta);
-            if (plan.n_seg == vitk::kMaxSegPerLaunch || plan.n_work + tiles > vitk::kMaxWorkPerLaunch) {
-                if (plan.n_seg == 0) return VIT_ERR_LIMIT;
-                break;
-            }
-            const int ls = plan.n_seg++;
-            plan.start[ls] = cu_seqlens[sg];
-            plan.len[ls] = len;
-            for (int t = 0; t < tiles; ++t) plan.work[plan.n_work++] = (ls << 16) | t;
-            ++pos;
-        }
-        if (plan.n_work > 0) {
-            vitk::attn_tc_kernel<<<plan.n_work * VIT_HEADS, vitk::kAttnThreads, vitk::kAttnSmem, s>>>(
-                tqkv.q, tqkv.kv, plan, static_cast<__nv_bfloat16 *>(out), status);
-            if (cudaGetLastError() != cudaSuccess) return VIT_ERR_CUDA;
-        }
-    }
-    return VIT_OK;
+    return launch_plans(plan, order, n_seg, cu_seqlens, tqkv, out, status, s);
 }
 
 }  // namespace vith

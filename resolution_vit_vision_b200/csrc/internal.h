@@ -38,6 +38,9 @@ int attn_make_maps(AttnMaps *m, const void *qkv, int64_t P);
 int attn_launch(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg, void *out, int32_t *status,
                 cudaStream_t s);
 
+// the FMA-pipe exponential of the attention softmax, elementwise (parity checks)
+int exp2_fma_launch(const float *x, float *y, int64_t n, cudaStream_t s);
+
 // ---- small kernels (misc.cu)
 int layernorm_launch(const float *X, const void *gamma, const void *beta, void *Y, int64_t rows, float eps,
                      const int32_t *out_row, cudaStream_t s);

@@ -185,8 +185,17 @@ __global__ void __launch_bounds__(kMropeThreads)
         if (n_runs > g.n) s_err = 1;
         int shift = 0, prev_end = 0;
         for (int k = 0; k < n_runs && !s_err; ++k) {
-            const int hh = g.h[k] >> 1, ww = g.w[k] >> 1;
-            const int n = g.t[k] * hh * ww;
+            // a grid is checked only when a run consumes it (unused trailing grids are ignored);
+            // every factor of a run's length is at most the prompt length, so each is bounded by
+            // L before the product is formed
+            const int64_t gt = g.t[k], gh = g.h[k], gw = g.w[k];
+            if (gt < 1 || gh < 2 || gw < 2 || (gh & 1) || (gw & 1) || gt > L || gh / 2 > L || gw / 2 > L ||
+                gt * (gh / 2) > L || gt * (gh / 2) * (gw / 2) > L) {
+                s_err = 1;
+                break;
+            }
+            const int hh = static_cast<int>(gh >> 1), ww = static_cast<int>(gw >> 1);
+            const int n = static_cast<int>(gt) * hh * ww;
             const int a = max(g.t[k], max(hh, ww));
             const int s = s_start[k];
             if (s < prev_end || static_cast<int64_t>(s) + n > L) { s_err = 1; break; }

@@ -7,7 +7,9 @@
 // that forbids device allocation after start-up, because cudaMalloc can synchronise the whole
 // device and can fail at run time. For them this file holds the activations of one encode in a
 // fixed, file-scope device array instead, sized for at most VIT_NOALLOC_MAX_PATCHES patches.
-// The array exists on every GPU that loads the library, from load until process exit.
+// The array exists on every GPU where the module holding it is loaded: from the first call on
+// that device (CUDA's default lazy module loading) or from context creation (eager loading),
+// until process exit.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -38,15 +40,22 @@ std::mutex g_setup_mu;
 unsigned char *g_scratch_dev[64] = {};   // device address of g_scratch, per device
 
 // Once per device, with that device current: look up the array's device address (host code may
-// not use the symbol itself as an address) and fill the rope cos/sin table it holds.
+// not use the symbol itself as an address) and fill the rope cos/sin table it holds. Under CUDA's
+// lazy module loading (the default) the address lookup is what loads this file's module on the
+// device, and with it allocates the array. The set-up waits for the table fill, so a later call on
+// any other stream finds the table complete.
 int setup_device(int dev, cudaStream_t s) {
     std::lock_guard<std::mutex> lock(g_setup_mu);
     if (g_scratch_dev[dev]) return VIT_OK;
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return VIT_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return VIT_ERR_CUDA;
+    }
     unsigned char *base = static_cast<unsigned char *>(p);
     const int rc = vith::rope_table_launch(reinterpret_cast<float *>(base + kOffCs), kMaxSide + 1, s);
     if (rc != VIT_OK) return rc;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return VIT_ERR_CUDA;
     g_scratch_dev[dev] = base;
     return VIT_OK;
 }
@@ -67,6 +76,9 @@ extern "C" int vit_encode_noalloc(const void *patches, const int32_t *grid_thw, 
     for (int i = 0; i < n_images; ++i) {
         const int t = grid_thw[3 * i], hh = grid_thw[3 * i + 1], ww = grid_thw[3 * i + 2];
         if (t < 1 || hh < 2 || ww < 2 || (hh & 1) || (ww & 1)) return VIT_ERR_GRID;
+        // each factor is bounded before the product is formed: t * hh * ww <= kMaxP follows
+        if (hh > kMaxSide || ww > kMaxSide || t > kMaxP / 4) return VIT_ERR_LIMIT;
+        if (static_cast<int64_t>(hh) * ww > kMaxP) return VIT_ERR_LIMIT;
         P += static_cast<int64_t>(t) * hh * ww;
         if (P > kMaxP) return VIT_ERR_LIMIT;   // more patches than the fixed scratch holds
     }

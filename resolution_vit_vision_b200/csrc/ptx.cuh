@@ -337,6 +337,34 @@ __device__ __forceinline__ void fadd2(float &a0, float &a1, float b0, float b1) 
         : "f"(b0), "f"(b1));
 }
 
+// 2^x0 and 2^x1 on the FMA pipe, without the MUFU: Cody-Waite range reduction x = j + f with
+// j = rint(x), read from the low mantissa bits of x + 1.5 * 2^23 (exact for |x| < 2^22), so
+// f = x - j is exact and lies in [-1/2, 1/2]; 2^f from a degree-3 polynomial, the minimax fit of
+// the relative error on [-1/2, 1/2] by the Remez exchange algorithm (csrc/fit_exp2_poly.py; max
+// relative error 7.5e-5 in float32); then j is added to the exponent field of 2^f. x is first
+// clamped to >= -127.5: there (and for every x < -127 with f < 0) the biased exponent would go
+// negative, and the final integer max turns those results into +0, so -inf gives exactly 0 and
+// results below 2^-126 are 0 or a subnormal below 2^-126.
+__device__ __forceinline__ void exp2_fma2(float &x0, float &x1) {
+    constexpr float kShift = 12582912.0f;              // 1.5 * 2^23
+    constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f, c2 = 0.2426111251115799f,
+                    c3 = 0.0551716685295105f;
+    x0 = fmaxf(x0, -127.5f);
+    x1 = fmaxf(x1, -127.5f);
+    float t0 = x0, t1 = x1;
+    fadd2(t0, t1, kShift, kShift);                     // kShift + rint(x)
+    float j0 = t0, j1 = t1;
+    fadd2(j0, j1, -kShift, -kShift);                   // rint(x)
+    float f0, f1, p0, p1;
+    ffma2(f0, f1, j0, j1, -1.0f, -1.0f, x0, x1);       // f = x - j, exact
+    ffma2(p0, p1, c3, c3, f0, f1, c2, c2);
+    ffma2(p0, p1, p0, p1, f0, f1, c1, c1);
+    ffma2(p0, p1, p0, p1, f0, f1, c0, c0);
+    // the low 9 bits of kShift's encoding are 0, so (bits(t) << 23) == j << 23 (mod 2^32)
+    x0 = __int_as_float(max(static_cast<int>(__float_as_uint(t0) << 23) + __float_as_int(p0), 0));
+    x1 = __int_as_float(max(static_cast<int>(__float_as_uint(t1) << 23) + __float_as_int(p1), 0));
+}
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

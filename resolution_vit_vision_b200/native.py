@@ -64,6 +64,7 @@ _SIGS = {
     "vit_op_layernorm": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_float, c_void_p, c_void_p]),
     "vit_op_attention": (c_int, [c_void_p, c_int64, c_i32p, c_int, c_void_p, c_void_p, c_void_p]),
     "vit_op_wait_selftest": (c_int, [c_void_p, c_int64, c_void_p]),
+    "vit_op_exp2_fma": (c_int, [c_void_p, c_void_p, c_int64, c_void_p]),
     "mrope_apply": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_int64, ctypes.c_double, c_i32p,
                             c_void_p]),
     "scatter_vision_tokens": (c_int, [c_void_p, c_int64, c_void_p, c_int64, c_int, c_void_p, c_int64, c_void_p,
@@ -305,6 +306,14 @@ def op_attention(qkv, cu_seqlens: Sequence[int], out, status=None, stream=None):
     check(lib().vit_op_attention(_ptr(qkv), qkv.shape[0], cu.ctypes.data_as(c_i32p), cu.shape[0] - 1, _ptr(out),
                                  _ptr(status), _stream(stream)), "vit_op_attention")
     return out
+
+
+def op_exp2_fma(x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The attention softmax's FMA-pipe exponential 2^x, elementwise on fp32 device tensors."""
+    assert x.dtype == torch.float32 and x.is_cuda and x.is_contiguous()
+    y = torch.empty_like(x) if y is None else y
+    check(lib().vit_op_exp2_fma(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "vit_op_exp2_fma")
+    return y
 
 
 def op_window_positions(grid_thw, patch_order: int, window: int, device="cuda", stream=None):

@@ -167,6 +167,20 @@ def make_f32(shape, seed: int, std: float = 1.0) -> np.ndarray:
     return (rng.standard_normal(shape, dtype=np.float32) * np.float32(std)).astype(np.float32)
 
 
+def device_normal_bf16(shape, seed: int, std: float = 1.0, device="cuda"):
+    """A seeded N(0, std) bf16 tensor drawn on the device (torch's generator), for inputs too
+    large to draw on the host; tests copy what the oracle needs back from it."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    rows = max(1, (1 << 28) // max(1, int(np.prod(shape[1:]))))   # bounded fp32 temporaries
+    for r0 in range(0, shape[0], rows):
+        r1 = min(shape[0], r0 + rows)
+        out[r0:r1] = (torch.randn((r1 - r0,) + tuple(shape[1:]), generator=g, device=device) * std).to(torch.bfloat16)
+    return out
+
+
 # ----------------------------------------------------------------------------------------------
 # M-RoPE prompts
 # ----------------------------------------------------------------------------------------------

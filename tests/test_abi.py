@@ -107,7 +107,9 @@ def test_mrope_rejects_bad_arguments(lib):
     from resolution_vit_vision_b200 import native as nv
     g = np.array([[1, 3, 4]], np.int32)
     assert lib.mrope_index(None, 5, None, 0, None, None, None, None) == nv.VIT_ERR_ARG
-    assert lib.mrope_index(ctypes.c_void_p(16), 5, nv._gp(g), 1, ctypes.c_void_p(16), None, None, None) == nv.VIT_ERR_GRID
+    # grid values are checked on the device and only for consumed grids: no host-side refusal
+    assert lib.mrope_index(ctypes.c_void_p(16), (1 << 30) + 1, nv._gp(g), 1, ctypes.c_void_p(16), None, None,
+                           None) == nv.VIT_ERR_LIMIT
     assert lib.mrope_index(ctypes.c_void_p(16), 5, None, 1, ctypes.c_void_p(16), None, None, None) == nv.VIT_ERR_ARG
     assert lib.mrope_index(ctypes.c_void_p(16), -1, None, 0, ctypes.c_void_p(16), None, None, None) == nv.VIT_ERR_ARG
 

@@ -158,6 +158,70 @@ def test_attention_varlen(lens):
     assert_attention_close(to_np(out), ref, np.abs(v).max(), f"attention {lens}")
 
 
+def test_attention_more_segments_than_one_launch():
+    # 700 segments: more than one launch's segment table holds, so the work is split across
+    # launches; lengths 0..40 (empty, tiny and ragged segments)
+    lens = np.random.Generator(np.random.PCG64(77)).integers(0, 41, size=700)
+    P = int(lens.sum())
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    qkv = _bits((P, 3840), 78, 1.0)
+    out = torch.full((P, 1280), float("nan"), dtype=torch.bfloat16, device=DEV)
+    st = _status()
+    nv.op_attention(bf16_bits_to_torch(qkv), cu, out, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    x = vo._f64(qkv)
+    q, k, v = (x[:, i * 1280:(i + 1) * 1280].reshape(P, 16, 80) for i in range(3))
+    segs = [(int(cu[i]), int(lens[i]), 0, 0) for i in range(len(lens)) if lens[i] > 0]
+    ref = vo.varlen_attention(q, k, v, segs)
+    assert_attention_close(to_np(out), ref, np.abs(v).max(), "attention, 700 segments")
+
+
+@pytest.mark.slow
+def test_attention_one_segment_across_launches():
+    # one segment longer than a launch's work table (4096 pairs of 128-query tiles): its query
+    # tiles continue in a second launch, which must still see every key of the segment. Inputs
+    # are drawn on the device (seeded); the oracle takes sampled query rows one by one against
+    # all keys, on four of the heads.
+    P = 4096 * 256 + 3000
+    qkv = syn.device_normal_bf16((P, 3840), 79, 1.0)
+    out = torch.full((P, 1280), float("nan"), dtype=torch.bfloat16, device=DEV)
+    st = _status()
+    nv.op_attention(qkv, np.array([0, P], np.int32), out, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rows = np.array([0, 1, 123457, 1048575, 1048576, 1048577, 1050000, P - 1])
+    for h in (0, 5, 10, 15):
+        q = to_np(qkv[rows, h * 80:(h + 1) * 80])
+        k = to_np(qkv[:, 1280 + h * 80:1280 + (h + 1) * 80])
+        v = to_np(qkv[:, 2560 + h * 80:2560 + (h + 1) * 80])
+        ref = vo.attention(q, k, v)
+        assert_attention_close(to_np(out[rows, h * 80:(h + 1) * 80]), ref, np.abs(v).max(),
+                               f"one {P}-row segment, head {h}")
+    del qkv, out
+    torch.cuda.empty_cache()
+
+
+def test_exp2_fma_dense_sweep():
+    # the FMA-pipe exponential of the softmax against the exact 2^x: relative error within the
+    # minimax bound (7.5e-5) plus float32 rounding wherever 2^x is a normal number, exactly 0 at
+    # and below -127.5 (masked scores are -inf), and nothing above 2^-126 in between
+    xs = np.concatenate([np.linspace(-140.0, 20.0, 4_000_001), np.arange(-130, 21, dtype=np.float64),
+                         np.arange(-130, 21) + 0.5, [-np.inf, -127.5, -126.0, 0.0, -0.0, 8.0]]).astype(np.float32)
+    x = torch.from_numpy(xs).to(DEV)
+    y = nv.op_exp2_fma(x).cpu().numpy().astype(np.float64)
+    ref = np.exp2(xs.astype(np.float64))
+    normal = xs >= -125.0            # results >= 2^-125: normal numbers whatever 2^f's exponent
+    rel = np.abs(y[normal] / ref[normal] - 1.0)
+    assert rel.max() <= 7.5e-5 + 4 * 2.0 ** -24, rel.max()
+    assert (y[xs <= -127.5] == 0.0).all()
+    mid = (xs > -127.5) & (xs < -125.0)
+    assert ((y[mid] >= 0.0) & (y[mid] <= 2.0 ** -124)).all()
+    assert np.isfinite(y).all() and (y >= 0).all()
+    # a smooth sweep: the polynomial's error matters, not a single point
+    assert rel.mean() < 5e-5
+
+
 def test_attention_large_scores():
     # sharply peaked softmax: scores of order 100 exercise the running-max rescale
     lens = [384]
@@ -201,17 +265,42 @@ def test_mrope_bit_exact(which):
     assert delta == rdelta
 
 
-@pytest.mark.parametrize("case", ["short", "long", "no_grid"])
+@pytest.mark.parametrize("case", ["short", "long", "no_grid", "odd_grid", "zero_t", "huge_grid"])
 def test_mrope_malformed_sets_status(case):
     if case == "short":
         ids, grids = syn.make_prompt([("image", 15)], 0), [[1, 8, 8]]
     elif case == "long":
         ids, grids = syn.make_prompt([("image", 17)], 0), [[1, 8, 8]]
-    else:
+    elif case == "no_grid":
         ids, grids = syn.make_prompt([("image", 16), ("image", 16)], 0), [[1, 8, 8]]
+    elif case == "odd_grid":      # a consumed grid with an odd side
+        ids, grids = syn.make_prompt([("image", 4)], 0), [[1, 3, 8]]
+    elif case == "zero_t":
+        ids, grids = syn.make_prompt([("image", 4)], 0), [[0, 4, 4]]
+    else:                         # factors whose product would overflow
+        ids, grids = syn.make_prompt([("image", 4)], 0), [[1 << 30, 1 << 30, 1 << 30]]
+    if case in ("odd_grid", "zero_t", "huge_grid"):
+        with pytest.raises(mo.MRopeError):
+            mo.mrope_index(ids, grids)
     got, delta, st = _mrope_gpu(ids, grids)
     assert st == nv.VIT_ERR_TOKENS
     assert (got == -7).all() and delta == -7      # nothing written
+
+
+def test_mrope_ignores_unused_trailing_grids():
+    # the oracle checks a grid only when a vision run consumes it; malformed grids after the
+    # last consumed one change nothing
+    ids = syn.make_prompt([("text", 7), ("image", 16), ("text", 9), ("video", 12), ("text", 3)], 21)
+    used = [[1, 8, 8], [3, 4, 4]]
+    ref, rdelta = mo.mrope_index(ids, used)
+    for tail in ([[1, 3, 8]], [[0, 4, 4], [1, 1 << 30, 1 << 30]], [[-5, 7, 9]]):
+        grids = np.array(used + tail, np.int32)
+        r2, d2 = mo.mrope_index(ids, grids)
+        np.testing.assert_array_equal(r2, ref)
+        got, delta, st = _mrope_gpu(ids, grids)
+        assert st == 0, tail
+        np.testing.assert_array_equal(got, ref)
+        assert delta == rdelta == d2
 
 
 def test_mrope_empty_prompt():
