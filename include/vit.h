@@ -82,6 +82,18 @@ typedef struct {
     const void *fc2_w, *fc2_b;     /* [1280, 5120], [1280]   */
 } vit_layer_w;
 
+/* The fp8 variant of one block's four linears ("Qwen2-VL-2B-Instruct -- LiteRT-LM", file table:
+ * the vision tower ships with 8-bit weights; correlation note: 0.90 with them). Codes: FP8 E4M3
+ * (OCP "e4m3fn": bias 7, max 448, no infinities), [out, in] row-major, one byte each; scales:
+ * fp32 [out], one power of two per output channel, weight = scale * code. vit_quantize_fp8 makes
+ * both from bf16 weights. All device pointers, 16-byte aligned. */
+typedef struct {
+    const void *qkv_q;  const float *qkv_s;    /* [3840, 1280], [3840] */
+    const void *proj_q; const float *proj_s;   /* [1280, 1280], [1280] */
+    const void *fc1_q;  const float *fc1_s;    /* [5120, 1280], [5120] */
+    const void *fc2_q;  const float *fc2_s;    /* [1280, 5120], [1280] */
+} vit_layer_fp8;
+
 typedef struct {
     int depth;                 /* number of ViT blocks, 1..64 (32 for Qwen2-VL)                  */
     int out_dim;               /* merger output width: a multiple of 16, 16..16384 (1536, 3584)  */
@@ -105,6 +117,15 @@ typedef struct {
     const uint8_t *full_attention; /* HOST [depth] or NULL; copied by vit_weights_create. With
                                       window > 0, block l attends over the whole frame where
                                       full_attention[l] != 0 (Qwen2.5-VL: l = 7, 15, 23, 31) */
+    /* HOST array [depth] or NULL (zero-initialised: the bf16 tower). Given, every block's four
+     * linears run as E4M3 products on the tensor cores: the input rows of each product are
+     * quantised at run time (E4M3 codes, one power-of-two scale per row, taken from the row's max
+     * |x|: the LayerNorm kernels emit them for QKV and fc1, a quantisation pass for out-proj and
+     * fc2), the accumulator is multiplied by the row's and the channel's scales, then the bias
+     * is added in fp32. The layers' qkv_w, proj_w, fc1_w and fc2_w may then be NULL. Everything
+     * else (LayerNorms, rope, attention, GELU, the fp32 residual stream, the patch embed and the
+     * merger) is as in the bf16 tower. Copied by vit_weights_create. */
+    const vit_layer_fp8 *fp8_layers;
 } vit_weights_desc;
 
 typedef struct vit_handle vit_handle;  /* validated weight view + workspace + device status word */
@@ -173,6 +194,13 @@ int vit_encode_host(const void *host_patches, const int32_t *grid_thw, int n_ima
 int mrope_index(const int32_t *input_ids, int64_t L, const int32_t *grid_thw, int n_grids,
                 int32_t *out, int32_t *delta, int32_t *dev_status, void *stream);
 
+/* E4M3 codes of bf16 rows with one power-of-two scale per row (the fp8 tower's weights: one row =
+ * one output channel). x: bf16 [rows, cols]; codes: [rows, cols] bytes; scales: fp32 [rows]. Row r
+ * with a = max |x[r]| gets scale 2^e, e the smallest integer with a <= 448 * 2^e but at least
+ * -126; codes[r][c] = x[r][c] / 2^e (exact) rounded to the nearest E4M3 value, ties to even.
+ * cols: a multiple of 8, 8..65536; rows >= 0; x and codes 16-byte aligned. Async on stream. */
+int vit_quantize_fp8(const void *x, int64_t rows, int cols, void *codes, float *scales, void *stream);
+
 /* ---- for callers that cannot allocate device memory ----------------------------------------
  * No counterpart on the pages: this is a deployment variant of vit_encode, not part of the method.
  * vit_encode keeps its activations in a workspace the handle grows with cudaMalloc. Callers whose
@@ -198,7 +226,8 @@ int mrope_index(const int32_t *input_ids, int64_t L, const int32_t *grid_thw, in
  *     order them. Nothing in the array needs clearing between calls: each buffer is fully
  *     written before it is read.
  *   - Arguments as for vit_encode; weights from vit_weights_create on the current device, made
- *     without windows (desc.window == 0; a windowed handle returns VIT_ERR_ARG). A grid row with
+ *     without windows and without fp8 layers (desc.window == 0, desc.fp8_layers == NULL; other
+ *     handles return VIT_ERR_ARG). A grid row with
  *     h or w above VIT_NOALLOC_MAX_PATCHES / 2, or t above VIT_NOALLOC_MAX_PATCHES / 4, returns
  *     VIT_ERR_LIMIT before any product of its values is formed.
  *     dev_status: int32 [1] device or NULL; a kernel wait that timed out writes VIT_ERR_TIMEOUT

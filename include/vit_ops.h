@@ -36,6 +36,19 @@ int vit_op_gemm(const void *A, const void *B, const void *bias, void *C, int64_t
                 int epilogue, const int32_t *pos, const float *rope_cs, int32_t *dev_status,
                 void *stream);
 
+/* The fp8 tower's product (vit.h, vit_layer_fp8): C = (a_scale[m] * b_scale[n]) * (A B^T)[m, n]
+ * (+ bias) with A E4M3 codes [M, K], B E4M3 codes [N, K] (one byte each), a_scale fp32 [M],
+ * b_scale fp32 [N] (16-byte aligned), the same epilogues as vit_op_gemm (the scales are applied
+ * to the fp32 accumulator first). Requirements as vit_op_gemm, and K % 16 == 0. */
+int vit_op_gemm_fp8(const void *A, const float *a_scale, const void *B, const float *b_scale, const void *bias,
+                    void *C, int64_t M, int N, int K, int epilogue, const int32_t *pos, const float *rope_cs,
+                    int32_t *dev_status, void *stream);
+
+/* LayerNorm of fp32 rows of 1280 (as vit_op_layernorm), the output row quantised as by
+ * vit_quantize_fp8: codes [rows, 1280] bytes, scales fp32 [rows] (one power of two per row). */
+int vit_op_layernorm_fp8(const float *X, const void *gamma, const void *beta, void *codes, float *scales,
+                         int64_t rows, float eps, void *stream);
+
 /* Rope table ("Qwen2-VL (Native-Resolution VLM)", Structure row 3, 2D RoPE; LiteRT-LM card,
  * Conversion notes: precomputed 2-D rope): cs[p][k] = (cos(p f_k), sin(p f_k)), f_k =
  * 10000^(-2k/40), k < 20, p < n_pos. cs: fp32 [n_pos * 40]. */

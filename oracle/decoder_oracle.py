@@ -16,7 +16,7 @@ Passages followed:
   Resolution VLM)" Structure table rows 6-10: the merged image tokens and the embedded text tokens
   form one sequence of the decoder's width.
 
-Readings of what the pages leave open (each is listed in the design doc):
+Readings of what the pages leave open:
 
 * head_dim = 2 * sum(sections); frequency j < head_dim / 2 is theta^(-2j / head_dim) and turns
   dims j and j + head_dim/2 as a pair (rotate-half, the decoder's 1-D convention), by the angle

@@ -14,7 +14,7 @@ Passages followed:
 * "Qwen2.5-VL-7B-Instruct" record: tokens per image = pixels / (28*28), i.e. one position per
   merged 2x2 group.
 
-Reading (the design doc lists it): walk the tokens with a cursor c = (largest id so far) + 1. Every
+Reading of the rule, which the pages leave open: walk the tokens with a cursor c = (largest id so far) + 1. Every
 token outside a vision run, vision_start/end included, gets (c, c, c) and advances c by one.
 A vision run starts right after a vision_start whose next token is the image or video id; it
 takes the next (t, h, w) from ``grid_thw`` (images and videos in appearance order) and must be

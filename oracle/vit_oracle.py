@@ -19,7 +19,7 @@ pages give it, with numpy's matmul as the only library primitive. Passages follo
   the patch embed is a Conv3d over 2 temporal frames; the 2x2 merge of raster-ordered patches is
   four strided slices, and ordering is irrelevant as long as each patch keeps its own 2-D rope.
 
-Readings of points the pages leave open (each is listed in the design doc):
+Readings of points the pages leave open:
 
 * pre-norm blocks, LayerNorm eps 1e-6 with gamma/beta, exact-erf GELU;
 * patch vector order (c, t, ph, pw), c-major: the Conv3d weight [1280, 3, 2, 14, 14] flattened;

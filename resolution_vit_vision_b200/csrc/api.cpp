@@ -74,8 +74,8 @@ namespace {
 
 const char *kProfNames[vith::kProfClasses] = {"patch_embed", "layernorm",  "qkv_rope",   "attention",
                                               "out_proj",    "fc1_gelu",   "fc2",        "merger_fc1",
-                                              "merger_fc2",  "positions",  "attention_window"};
-enum ProfClass { P_PE, P_LN, P_QKV, P_ATT, P_PROJ, P_FC1, P_FC2, P_M0, P_M2, P_POS, P_WATT };
+                                              "merger_fc2",  "positions",  "attention_window", "quantize_fp8"};
+enum ProfClass { P_PE, P_LN, P_QKV, P_ATT, P_PROJ, P_FC1, P_FC2, P_M0, P_M2, P_POS, P_WATT, P_Q8 };
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -160,6 +160,9 @@ int ensure_workspace(vit_handle *h, int64_t P) {
     const size_t oOs = take(static_cast<size_t>(Pn / 4 + 1) * out_dim * 2);
     const size_t oCs = take(static_cast<size_t>(VIT_MAX_SIDE) * 40 * 4);
     const size_t oSt = take(256);
+    const bool f8 = !h->fp8.empty();
+    const size_t oQ8 = f8 ? take(static_cast<size_t>(Pn) * VIT_MLP) : 0;
+    const size_t oS8 = f8 ? take(static_cast<size_t>(Pn) * 4) : 0;
     if (h->ws) {
         cudaDeviceSynchronize();
         graph_clear(h);           // recorded graphs point into the old workspace
@@ -187,6 +190,8 @@ int ensure_workspace(vit_handle *h, int64_t P) {
     h->out_stage = b + oOs;
     h->rope_cs = reinterpret_cast<float *>(b + oCs);
     h->status = reinterpret_cast<int32_t *>(b + oSt);
+    h->Q8 = f8 ? b + oQ8 : nullptr;
+    h->S8 = f8 ? reinterpret_cast<float *>(b + oS8) : nullptr;
     h->rope_ready = false;
     if (cudaMemset(h->status, 0, 4) != cudaSuccess) return VIT_ERR_CUDA;
     return VIT_OK;
@@ -242,7 +247,8 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
         patches = h->F;
     }
 
-    CUtensorMap mPatch, mH, mF, mH4, mF4;
+    const bool f8 = !h->fp8.empty();
+    CUtensorMap mPatch, mH, mF, mH4, mF4, mQ8w, mQ8m;   // mQ8w / mQ8m: E4M3 rows of 1280 / 5120
     vith::WinMaps mWin;
     const int n_windows = window > 0 ? vith::window_count(grid, n_images, window) : 0;
     vith::AttnMaps mQKV;
@@ -253,6 +259,10 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
     VIT_TRY(vith::gemm_make_a_map(&mH4, h->H, M4, VIT_MERGE_DIM));
     VIT_TRY(vith::gemm_make_a_map(&mF4, h->F, M4, VIT_MERGE_DIM));
     VIT_TRY(vith::attn_make_maps(&mQKV, h->QKV, P));
+    if (f8) {
+        VIT_TRY(vith::gemm_make_a_map(&mQ8w, h->Q8, P, VIT_WIDTH, true));
+        VIT_TRY(vith::gemm_make_a_map(&mQ8m, h->Q8, P, VIT_MLP, true));
+    }
     CUtensorMap cX, cQKV, cF, cF4, cOut;
     VIT_TRY(vith::gemm_make_c_map(&cX, h->X, P, VIT_WIDTH, VIT_EPI_ADD_F32));
     VIT_TRY(vith::gemm_make_c_map(&cQKV, h->QKV, P, 3 * VIT_WIDTH, VIT_EPI_QKV_ROPE));
@@ -269,15 +279,18 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
     for (int l = 0; l < d.depth; ++l) {
         const vit_layer_w &L = h->layers[l];
         const vith::LayerMaps &lm = h->maps[l];
+        const vit_layer_fp8 *L8 = f8 ? &h->fp8[l] : nullptr;
         {
             ProfScope ps(h, s, P_LN);
-            VIT_TRY(vith::layernorm_launch(h->X, L.ln1_w, L.ln1_b, h->H, P, d.ln_eps, nullptr, s));
+            if (f8) VIT_TRY(vith::layernorm_fp8_launch(h->X, L.ln1_w, L.ln1_b, h->Q8, h->S8, P, d.ln_eps, s));
+            else VIT_TRY(vith::layernorm_launch(h->X, L.ln1_w, L.ln1_b, h->H, P, d.ln_eps, nullptr, s));
             ++nl;
         }
         {
             ProfScope ps(h, s, P_QKV);
-            VIT_TRY(vith::gemm_launch(mH, lm.qkv, cQKV, L.qkv_b, P, 3 * VIT_WIDTH, VIT_WIDTH, VIT_EPI_QKV_ROPE,
-                                      h->pos, h->rope_cs, h->status, s));
+            VIT_TRY(vith::gemm_launch(f8 ? mQ8w : mH, lm.qkv, cQKV, L.qkv_b, P, 3 * VIT_WIDTH, VIT_WIDTH,
+                                      VIT_EPI_QKV_ROPE, h->pos, h->rope_cs, h->status, s, f8 ? h->S8 : nullptr,
+                                      f8 ? L8->qkv_s : nullptr));
             ++nl;
         }
         if (window == 0 || h->full_attention[l]) {
@@ -293,27 +306,41 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
             VIT_TRY(vith::attn_launch(mQKV, cu_win.data(), static_cast<int>(cu_win.size()) - 1, h->H, h->status, s));
             ++nl;
         }
+        if (f8) {
+            ProfScope ps(h, s, P_Q8);
+            VIT_TRY(vith::quantize_rows_launch(h->H, P, VIT_WIDTH, h->Q8, h->S8, s));
+            ++nl;
+        }
         {
             ProfScope ps(h, s, P_PROJ);
-            VIT_TRY(vith::gemm_launch(mH, lm.proj, cX, L.proj_b, P, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32, nullptr,
-                                      nullptr, h->status, s));
+            VIT_TRY(vith::gemm_launch(f8 ? mQ8w : mH, lm.proj, cX, L.proj_b, P, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32,
+                                      nullptr, nullptr, h->status, s, f8 ? h->S8 : nullptr,
+                                      f8 ? L8->proj_s : nullptr));
             ++nl;
         }
         {
             ProfScope ps(h, s, P_LN);
-            VIT_TRY(vith::layernorm_launch(h->X, L.ln2_w, L.ln2_b, h->H, P, d.ln_eps, nullptr, s));
+            if (f8) VIT_TRY(vith::layernorm_fp8_launch(h->X, L.ln2_w, L.ln2_b, h->Q8, h->S8, P, d.ln_eps, s));
+            else VIT_TRY(vith::layernorm_launch(h->X, L.ln2_w, L.ln2_b, h->H, P, d.ln_eps, nullptr, s));
             ++nl;
         }
         {
             ProfScope ps(h, s, P_FC1);
-            VIT_TRY(vith::gemm_launch(mH, lm.fc1, cF, L.fc1_b, P, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16, nullptr,
-                                      nullptr, h->status, s));
+            VIT_TRY(vith::gemm_launch(f8 ? mQ8w : mH, lm.fc1, cF, L.fc1_b, P, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16,
+                                      nullptr, nullptr, h->status, s, f8 ? h->S8 : nullptr,
+                                      f8 ? L8->fc1_s : nullptr));
+            ++nl;
+        }
+        if (f8) {
+            ProfScope ps(h, s, P_Q8);
+            VIT_TRY(vith::quantize_rows_launch(h->F, P, VIT_MLP, h->Q8, h->S8, s));
             ++nl;
         }
         {
             ProfScope ps(h, s, P_FC2);
-            VIT_TRY(vith::gemm_launch(mF, lm.fc2, cX, L.fc2_b, P, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32, nullptr,
-                                      nullptr, h->status, s));
+            VIT_TRY(vith::gemm_launch(f8 ? mQ8m : mF, lm.fc2, cX, L.fc2_b, P, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32,
+                                      nullptr, nullptr, h->status, s, f8 ? h->S8 : nullptr,
+                                      f8 ? L8->fc2_s : nullptr));
             ++nl;
         }
     }
@@ -455,9 +482,21 @@ int vit_weights_create(const vit_weights_desc *d, vit_handle **out) {
         if (p && !aligned16(p)) return VIT_ERR_ALIGN;
     for (int l = 0; l < d->depth; ++l) {
         const vit_layer_w &L = d->layers[l];
-        const void *lr[] = {L.ln1_w, L.qkv_w, L.proj_w, L.ln2_w, L.fc1_w, L.fc2_w};
+        const void *lr[] = {L.ln1_w, L.ln2_w};
         for (const void *p : lr)
             if (!p) return VIT_ERR_ARG;
+        if (d->fp8_layers) {   // the E4M3 codes and scales replace the four bf16 block linears
+            const vit_layer_fp8 &Q = d->fp8_layers[l];
+            const void *q[] = {Q.qkv_q, Q.qkv_s, Q.proj_q, Q.proj_s, Q.fc1_q, Q.fc1_s, Q.fc2_q, Q.fc2_s};
+            for (const void *p : q) {
+                if (!p) return VIT_ERR_ARG;
+                if (!aligned16(p)) return VIT_ERR_ALIGN;
+            }
+        } else {
+            const void *w[] = {L.qkv_w, L.proj_w, L.fc1_w, L.fc2_w};
+            for (const void *p : w)
+                if (!p) return VIT_ERR_ARG;
+        }
         const void *la[] = {L.ln1_w, L.ln1_b, L.qkv_w, L.qkv_b, L.proj_w, L.proj_b,
                             L.ln2_w, L.ln2_b, L.fc1_w, L.fc1_b, L.fc2_w, L.fc2_b};
         for (const void *p : la)
@@ -474,6 +513,8 @@ int vit_weights_create(const vit_weights_desc *d, vit_handle **out) {
     if (d->window > 0 && d->full_attention)
         for (int l = 0; l < d->depth; ++l) h->full_attention[l] = d->full_attention[l] ? 1 : 0;
     h->desc.full_attention = nullptr;
+    if (d->fp8_layers) h->fp8.assign(d->fp8_layers, d->fp8_layers + d->depth);
+    h->desc.fp8_layers = nullptr;
     cudaGetDevice(&h->device);
     h->maps.resize(d->depth);
     rc = vith::gemm_make_b_map(&h->pe_map, d->pe_w, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32);
@@ -482,10 +523,15 @@ int vit_weights_create(const vit_weights_desc *d, vit_handle **out) {
     for (int l = 0; l < d->depth && rc == VIT_OK; ++l) {
         const vit_layer_w &L = h->layers[l];
         vith::LayerMaps &m = h->maps[l];
-        rc = vith::gemm_make_b_map(&m.qkv, L.qkv_w, 3 * VIT_WIDTH, VIT_WIDTH, VIT_EPI_QKV_ROPE);
-        if (rc == VIT_OK) rc = vith::gemm_make_b_map(&m.proj, L.proj_w, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32);
-        if (rc == VIT_OK) rc = vith::gemm_make_b_map(&m.fc1, L.fc1_w, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16);
-        if (rc == VIT_OK) rc = vith::gemm_make_b_map(&m.fc2, L.fc2_w, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32);
+        const bool f8 = !h->fp8.empty();
+        const vit_layer_fp8 *Q = f8 ? &h->fp8[l] : nullptr;
+        rc = vith::gemm_make_b_map(&m.qkv, f8 ? Q->qkv_q : L.qkv_w, 3 * VIT_WIDTH, VIT_WIDTH, VIT_EPI_QKV_ROPE, f8);
+        if (rc == VIT_OK)
+            rc = vith::gemm_make_b_map(&m.proj, f8 ? Q->proj_q : L.proj_w, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32, f8);
+        if (rc == VIT_OK)
+            rc = vith::gemm_make_b_map(&m.fc1, f8 ? Q->fc1_q : L.fc1_w, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16, f8);
+        if (rc == VIT_OK)
+            rc = vith::gemm_make_b_map(&m.fc2, f8 ? Q->fc2_q : L.fc2_w, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32, f8);
     }
     if (rc != VIT_OK) return rc;
     *out = h.release();
@@ -615,6 +661,40 @@ int vit_op_gemm(const void *A, const void *B, const void *bias, void *C, int64_t
     if (rc != VIT_OK) return rc;
     return vith::gemm_launch(ta, tb, tc, bias, M, N, K, epilogue, pos, rope_cs, dev_status,
                              static_cast<cudaStream_t>(stream));
+}
+
+int vit_op_gemm_fp8(const void *A, const float *a_scale, const void *B, const float *b_scale, const void *bias,
+                    void *C, int64_t M, int N, int K, int epilogue, const int32_t *pos, const float *rope_cs,
+                    int32_t *dev_status, void *stream) {
+    if (!A || !B || !C || !a_scale || !b_scale || M < 1 || N < 16 || (N % 16) != 0 || K < 16 || (K % 16) != 0)
+        return VIT_ERR_ARG;
+    if (epilogue < VIT_EPI_STORE_F32 || epilogue > VIT_EPI_QKV_ROPE) return VIT_ERR_ARG;
+    if (epilogue == VIT_EPI_QKV_ROPE && (N != 3 * VIT_WIDTH || !pos || !rope_cs)) return VIT_ERR_ARG;
+    if (M > (int64_t(1) << 30)) return VIT_ERR_LIMIT;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(C) || !aligned16(b_scale) || (bias && !aligned16(bias)))
+        return VIT_ERR_ALIGN;
+    CUtensorMap ta, tb, tc;
+    int rc = vith::gemm_make_a_map(&ta, A, M, K, true);
+    if (rc == VIT_OK) rc = vith::gemm_make_b_map(&tb, B, N, K, epilogue, true);
+    if (rc == VIT_OK) rc = vith::gemm_make_c_map(&tc, C, M, N, epilogue);
+    if (rc != VIT_OK) return rc;
+    return vith::gemm_launch(ta, tb, tc, bias, M, N, K, epilogue, pos, rope_cs, dev_status,
+                             static_cast<cudaStream_t>(stream), a_scale, b_scale);
+}
+
+int vit_op_layernorm_fp8(const float *X, const void *gamma, const void *beta, void *codes, float *scales,
+                         int64_t rows, float eps, void *stream) {
+    if (!X || !gamma || !codes || !scales || rows < 0 || !(eps > 0.0f)) return VIT_ERR_ARG;
+    if (!aligned16(X) || !aligned16(codes) || !aligned16(gamma) || (beta && !aligned16(beta))) return VIT_ERR_ALIGN;
+    return vith::layernorm_fp8_launch(X, gamma, beta, codes, scales, rows, eps, static_cast<cudaStream_t>(stream));
+}
+
+int vit_quantize_fp8(const void *x, int64_t rows, int cols, void *codes, float *scales, void *stream) {
+    if (rows < 0 || cols < 8 || cols > 65536 || (cols % 8) != 0) return VIT_ERR_ARG;
+    if (rows > 0 && (!x || !codes || !scales)) return VIT_ERR_ARG;
+    if (rows > (int64_t(1) << 31)) return VIT_ERR_LIMIT;
+    if (rows > 0 && (!aligned16(x) || !aligned16(codes))) return VIT_ERR_ALIGN;
+    return vith::quantize_rows_launch(x, rows, cols, codes, scales, static_cast<cudaStream_t>(stream));
 }
 
 int vit_op_rope_table(float *cs, int n_pos, void *stream) {

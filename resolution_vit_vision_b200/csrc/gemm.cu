@@ -19,6 +19,11 @@
 //               GELU / 2-D rope, then the tile leaves through a double-buffered swizzled shared
 //               staging chunk and a TMA store -- or a TMA reduce-add into the fp32 residual
 //               stream, so the residual update never reads the residual into the SM.
+// The same kernel runs the fp8 tower's products (F8 = true): A and B are E4M3 codes with a
+// power-of-two scale per row of A and per row of B ("Qwen2-VL-2B-Instruct -- LiteRT-LM", file
+// table: an 8-bit vision tower); a 128-byte k-block then holds 128 elements instead of 64, the
+// tensor core runs kind::f8f6f4 (K = 32 per instruction) at twice the bf16 rate, and the epilogue
+// multiplies every accumulator by its row's and column's scales before the bias.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -48,6 +53,8 @@ struct GemmShape {
 
 struct GemmParams {
     const __nv_bfloat16 *bias;
+    const float *a_scale;             // F8 only: [M] power-of-two scale of each row of A
+    const float *b_scale;             // F8 only: [N] scale of each row of B (output column)
     const int32_t *pos;
     const float2 *rope_cs;
     int32_t *status;
@@ -100,6 +107,23 @@ __device__ __forceinline__ void add_bias(float *v, const __nv_bfloat16 *bias, in
     }
 }
 
+// v[j] *= sa * b_scale[col0 + j] (the fp8 products' dequantisation; b_scale 16-byte aligned,
+// col0 a multiple of 4), columns >= N skipped
+template <int NV>
+__device__ __forceinline__ void scale_cols(float *v, float sa, const float *b_scale, int col0, int N) {
+#pragma unroll
+    for (int q = 0; q < NV / 4; ++q) {
+        if (col0 + 4 * q < N) {
+            const float4 b = __ldg(reinterpret_cast<const float4 *>(b_scale + col0) + q);
+            float s0, s1, s2, s3;
+            fmul2(s0, s1, sa, sa, b.x, b.y);
+            fmul2(s2, s3, sa, sa, b.z, b.w);
+            fmul2(v[4 * q], v[4 * q + 1], v[4 * q], v[4 * q + 1], s0, s1);
+            fmul2(v[4 * q + 2], v[4 * q + 3], v[4 * q + 2], v[4 * q + 3], s2, s3);
+        }
+    }
+}
+
 // Writes one thread's row r of 128 bytes (eight 16-byte pieces) into a 128B-swizzled staging
 // chunk: piece q lands at piece q ^ (r % 8), the layout a SWIZZLE_128B TMA box expects.
 __device__ __forceinline__ void stage_row128(uint8_t *stg, int r, const uint32_t *w) {
@@ -131,7 +155,12 @@ __device__ __forceinline__ void rope_head(float *v, int hw, const float2 *cs) {
     }
 }
 
-template <int BN, int EPI>
+// instruction descriptor of kind::f8f6f4 with E4M3 A and B (format code 0), fp32 D
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+template <int BN, int EPI, bool F8>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                    const __grid_constant__ CUtensorMap tmc, GemmParams p) {
@@ -189,8 +218,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (!mbar_wait(empty + stage, phase ^ 1u, wc)) goto producer_done;
                     const uint32_t bar0 = cluster_addr(full + stage, 0);
                     if (rank == 0) mbar_expect_tx(full + stage, 2 * (S::A_BYTES + S::B_BYTES));
-                    tma_load_2d_pair(sA + stage * S::A_BYTES, &tma, bar0, kb * kBK, m0);
-                    tma_load_2d_pair(sB + stage * S::B_BYTES, &tmb, bar0, kb * kBK, n0);
+                    // a k-block is 128 bytes of each row: 64 bf16 or 128 E4M3 elements
+                    const int kx = kb * (F8 ? 2 * kBK : kBK);
+                    tma_load_2d_pair(sA + stage * S::A_BYTES, &tma, bar0, kx, m0);
+                    tma_load_2d_pair(sB + stage * S::B_BYTES, &tmb, bar0, kx, n0);
                     if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -198,7 +229,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
-            constexpr uint32_t idesc = idesc_bf16(2 * kBM, BN, false, false);
+            constexpr uint32_t idesc = F8 ? idesc_e4m3(2 * kBM, BN) : idesc_bf16(2 * kBM, BN, false, false);
             int stage = 0;
             uint32_t phase = 0;
             int local = 0;
@@ -215,11 +246,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t a_addr = smem_u32(sA + stage * S::A_BYTES);
                     const uint32_t b_addr = smem_u32(sB + stage * S::B_BYTES);
 #pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k) {
-                        // +32 bytes per 16-element K step inside the 128-byte swizzle atom
+                    for (int k = 0; k < 4; ++k) {
+                        // +32 bytes per K step (16 bf16 or 32 E4M3) inside the 128-byte swizzle atom
                         const uint64_t da = smem_desc(a_addr + k * 32, 16, 1024, kSwizzle128B);
                         const uint64_t db = smem_desc(b_addr + k * 32, 16, 1024, kSwizzle128B);
-                        mma_bf16_ss_pair(d_tmem, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+                        if (F8) mma_e4m3_ss_pair(d_tmem, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+                        else mma_bf16_ss_pair(d_tmem, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
                     }
                     mma_commit_pair(empty + stage, 0x3);
                     if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
@@ -272,8 +304,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 80; ++j) v[j] = __uint_as_float(u[j]);
                     const int col0 = n0 + hh * 80;
-                    add_bias<80>(v, p.bias, col0, p.N);
                     const int row = m0 + r;
+                    if (F8) scale_cols<80>(v, row < p.M ? __ldg(p.a_scale + row) : 0.0f, p.b_scale, col0, p.N);
+                    add_bias<80>(v, p.bias, col0, p.N);
                     if (col0 < 2 * VIT_WIDTH) rope_head(v, row < p.M ? p.pos[row] : 0, p.rope_cs);
                     uint8_t *stg = stage_acquire();
                     // five 32-byte-swizzled boxes of 16 columns: the 16-byte half h of row r goes
@@ -310,6 +343,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         float v[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(u[j]);
+                        if (F8) scale_cols<32>(v, m0 + r < p.M ? __ldg(p.a_scale + m0 + r) : 0.0f, p.b_scale, col0, p.N);
                         add_bias<32>(v, p.bias, col0, p.N);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(v[j]);
@@ -339,6 +373,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         float v[64];
 #pragma unroll
                         for (int j = 0; j < 64; ++j) v[j] = __uint_as_float(u[j]);
+                        if (F8) scale_cols<64>(v, m0 + r < p.M ? __ldg(p.a_scale + m0 + r) : 0.0f, p.b_scale, col0, p.N);
                         add_bias<64>(v, p.bias, col0, p.N);
                         uint32_t w[32];
 #pragma unroll
@@ -376,13 +411,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 namespace vith {
 
-int gemm_make_a_map(CUtensorMap *map, const void *A, int64_t M, int K) {
+int gemm_make_a_map(CUtensorMap *map, const void *A, int64_t M, int K, bool f8) {
+    // 128-byte boxes along K: 64 bf16 or 128 E4M3 codes
+    if (f8)
+        return tmap_2d(map, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, static_cast<uint64_t>(K), 2 * vitk::kBK,
+                       vitk::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
     return tmap_2d(map, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, static_cast<uint64_t>(K) * 2, vitk::kBK,
                    vitk::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue) {
+int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue, bool f8) {
     const uint32_t bn = (epilogue == VIT_EPI_QKV_ROPE) ? 240 : 256;   // each CTA of a pair loads half
+    if (f8)
+        return tmap_2d(map, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, static_cast<uint64_t>(K), 2 * vitk::kBK,
+                       bn / 2, CU_TENSOR_MAP_SWIZZLE_128B);
     return tmap_2d(map, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, N, static_cast<uint64_t>(K) * 2, vitk::kBK, bn / 2,
                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
@@ -402,7 +444,7 @@ int gemm_make_c_map(CUtensorMap *map, void *C, int64_t M, int N, int epilogue) {
     }
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool F8>
 static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc, const vitk::GemmParams &p,
                       cudaStream_t s) {
     using S = vitk::GemmShape<BN>;
@@ -410,7 +452,7 @@ static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtens
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !configured[dev]) {
-        if (cudaFuncSetAttribute(vitk::gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM) !=
+        if (cudaFuncSetAttribute(vitk::gemm_tc_kernel<BN, EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM) !=
             cudaSuccess)
             return VIT_ERR_CUDA;
         if (dev < 64) configured[dev] = true;
@@ -430,7 +472,7 @@ static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtens
     if (dev < 64 && max_clusters[dev] == 0) {
         cfg.gridDim = dim3(2 * 74);
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, vitk::gemm_tc_kernel<BN, EPI>, &cfg) != cudaSuccess || n < 1) {
+        if (cudaOccupancyMaxActiveClusters(&n, vitk::gemm_tc_kernel<BN, EPI, F8>, &cfg) != cudaSuccess || n < 1) {
             cudaGetLastError();
             n = device_sm_count() / 2;
         }
@@ -439,16 +481,20 @@ static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtens
     const int total = p.m_tiles * p.n_tiles;
     const int pairs = dev < 64 ? max_clusters[dev] : device_sm_count() / 2;
     cfg.gridDim = dim3(2 * (total < pairs ? total : pairs));
-    if (cudaLaunchKernelEx(&cfg, vitk::gemm_tc_kernel<BN, EPI>, ta, tb, tc, p) != cudaSuccess) return VIT_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, vitk::gemm_tc_kernel<BN, EPI, F8>, ta, tb, tc, p) != cudaSuccess) return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 
 int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc, const void *bias, int64_t M,
                 int N, int K, int epilogue, const int32_t *pos, const float *rope_cs, int32_t *status,
-                cudaStream_t s) {
+                cudaStream_t s, const float *a_scale, const float *b_scale) {
     if (M <= 0) return VIT_OK;
+    const bool f8 = a_scale != nullptr;
+    if (f8 && (!b_scale || K % 16)) return VIT_ERR_ARG;
     vitk::GemmParams p{};
     p.bias = static_cast<const __nv_bfloat16 *>(bias);
+    p.a_scale = a_scale;
+    p.b_scale = b_scale;
     p.pos = pos;
     p.rope_cs = reinterpret_cast<const float2 *>(rope_cs);
     p.status = status;
@@ -456,23 +502,29 @@ int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap 
     p.N = N;
     p.K = K;
     p.m_tiles = static_cast<int>((M + 2 * vitk::kBM - 1) / (2 * vitk::kBM));
-    p.k_blocks = (K + vitk::kBK - 1) / vitk::kBK;
+    const int kblk = f8 ? 2 * vitk::kBK : vitk::kBK;   // elements per 128-byte k-block
+    p.k_blocks = (K + kblk - 1) / kblk;
     switch (epilogue) {
         case VIT_EPI_QKV_ROPE:
             p.n_tiles = N / 240;
-            return launch_one<240, VIT_EPI_QKV_ROPE>(ta, tb, tc, p, s);
+            return f8 ? launch_one<240, VIT_EPI_QKV_ROPE, true>(ta, tb, tc, p, s)
+                      : launch_one<240, VIT_EPI_QKV_ROPE, false>(ta, tb, tc, p, s);
         case VIT_EPI_STORE_F32:
             p.n_tiles = (N + 255) / 256;
-            return launch_one<256, VIT_EPI_STORE_F32>(ta, tb, tc, p, s);
+            return f8 ? launch_one<256, VIT_EPI_STORE_F32, true>(ta, tb, tc, p, s)
+                      : launch_one<256, VIT_EPI_STORE_F32, false>(ta, tb, tc, p, s);
         case VIT_EPI_ADD_F32:
             p.n_tiles = (N + 255) / 256;
-            return launch_one<256, VIT_EPI_ADD_F32>(ta, tb, tc, p, s);
+            return f8 ? launch_one<256, VIT_EPI_ADD_F32, true>(ta, tb, tc, p, s)
+                      : launch_one<256, VIT_EPI_ADD_F32, false>(ta, tb, tc, p, s);
         case VIT_EPI_STORE_BF16:
             p.n_tiles = (N + 255) / 256;
-            return launch_one<256, VIT_EPI_STORE_BF16>(ta, tb, tc, p, s);
+            return f8 ? launch_one<256, VIT_EPI_STORE_BF16, true>(ta, tb, tc, p, s)
+                      : launch_one<256, VIT_EPI_STORE_BF16, false>(ta, tb, tc, p, s);
         case VIT_EPI_GELU_BF16:
             p.n_tiles = (N + 255) / 256;
-            return launch_one<256, VIT_EPI_GELU_BF16>(ta, tb, tc, p, s);
+            return f8 ? launch_one<256, VIT_EPI_GELU_BF16, true>(ta, tb, tc, p, s)
+                      : launch_one<256, VIT_EPI_GELU_BF16, false>(ta, tb, tc, p, s);
         default:
             return VIT_ERR_ARG;
     }

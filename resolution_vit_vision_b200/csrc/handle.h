@@ -13,14 +13,15 @@ namespace vith {
 struct LayerMaps {
     CUtensorMap qkv, proj, fc1, fc2;
 };
-constexpr int kProfClasses = 11;
+constexpr int kProfClasses = 12;
 }  // namespace vith
 
 struct vit_handle {
     vit_weights_desc desc{};
     std::vector<vit_layer_w> layers;
     std::vector<uint8_t> full_attention;   // [depth], windowed handles only
-    std::vector<vith::LayerMaps> maps;
+    std::vector<vit_layer_fp8> fp8;        // [depth] when the block linears run in E4M3, else empty
+    std::vector<vith::LayerMaps> maps;     // of the bf16 weights, or of the E4M3 codes
     CUtensorMap pe_map{}, m0_map{}, m2_map{};
     int device = 0;
 
@@ -36,6 +37,8 @@ struct vit_handle {
     int32_t *pos = nullptr;        // [P]
     int32_t *merge_row = nullptr;  // [P]
     int32_t *win_tab = nullptr;    // [2 * (P/4 + 1)] (first row, rows) per attention window
+    void *Q8 = nullptr;            // fp8 handles: E4M3 codes of a product's input rows [P, <= 5120]
+    float *S8 = nullptr;           // fp8 handles: their per-row scales [P]
     void *patch_stage = nullptr;   // bf16 [P, 1176] (vit_encode_host)
     void *out_stage = nullptr;     // bf16 [P/4, out_dim] (vit_encode_host)
     float *rope_cs = nullptr;      // [VIT_MAX_SIDE][20][2]

@@ -21,13 +21,16 @@ int device_sm_count();
 int check_device();   // VIT_OK when the current device is sm_100
 
 // ---- GEMM (gemm.cu). A bf16 [M, K], B bf16 [N, K]. The B map may be prebuilt (weights).
-int gemm_make_a_map(CUtensorMap *map, const void *A, int64_t M, int K);
-int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue);
+// f8: E4M3 codes (one byte per element) instead of bf16
+int gemm_make_a_map(CUtensorMap *map, const void *A, int64_t M, int K, bool f8 = false);
+int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue, bool f8 = false);
 // C [M, N]: fp32 for STORE_F32 / ADD_F32 (the output is written, or added, by TMA), else bf16
 int gemm_make_c_map(CUtensorMap *map, void *C, int64_t M, int N, int epilogue);
+// a_scale != NULL selects the E4M3 product: A and B are codes (maps made with f8), a_scale [M] and
+// b_scale [N] their per-row power-of-two scales, applied to the accumulator before the bias
 int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc, const void *bias, int64_t M,
                 int N, int K, int epilogue, const int32_t *pos, const float *rope_cs, int32_t *status,
-                cudaStream_t s);
+                cudaStream_t s, const float *a_scale = nullptr, const float *b_scale = nullptr);
 
 // ---- attention (attention.cu). qkv bf16 [P, 3840].
 struct AttnMaps {
@@ -40,6 +43,11 @@ int attn_launch(const AttnMaps &tqkv, const int32_t *cu_seqlens, int n_seg, void
 
 // the FMA-pipe exponential of the attention softmax, elementwise (parity checks)
 int exp2_fma_launch(const float *x, float *y, int64_t n, cudaStream_t s);
+
+// ---- E4M3 quantisation (fp8.cu): per-row power-of-two scales, codes rounded to nearest even
+int quantize_rows_launch(const void *x, int64_t rows, int cols, void *codes, float *scales, cudaStream_t s);
+int layernorm_fp8_launch(const float *X, const void *gamma, const void *beta, void *codes, float *scales,
+                         int64_t rows, float eps, cudaStream_t s);
 
 // ---- small kernels (misc.cu)
 int layernorm_launch(const float *X, const void *gamma, const void *beta, void *Y, int64_t rows, float eps,

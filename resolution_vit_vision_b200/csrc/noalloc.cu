@@ -71,7 +71,7 @@ int setup_device(int dev, cudaStream_t s) {
 extern "C" int vit_encode_noalloc(const void *patches, const int32_t *grid_thw, int n_images, vit_handle *h,
                                   void *out, int32_t *dev_status, void *stream) {
     if (!patches || !h || !out || !grid_thw || n_images < 1 || n_images > VIT_MAX_IMAGES) return VIT_ERR_ARG;
-    if (h->desc.window != 0) return VIT_ERR_ARG;   // windowed towers: vit_encode only
+    if (h->desc.window != 0 || !h->fp8.empty()) return VIT_ERR_ARG;   // windowed / fp8 towers: vit_encode only
     int64_t P = 0;
     for (int i = 0; i < n_images; ++i) {
         const int t = grid_thw[3 * i], hh = grid_thw[3 * i + 1], ww = grid_thw[3 * i + 2];

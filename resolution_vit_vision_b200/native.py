@@ -30,12 +30,20 @@ class VitLayerW(ctypes.Structure):
     _fields_ = [(k, c_void_p) for k in syn.LAYER_KEYS]
 
 
+FP8_LINEARS = ("qkv", "proj", "fc1", "fc2")
+
+
+class VitLayerFp8(ctypes.Structure):
+    _fields_ = [(f"{k}_{x}", c_void_p) for k in FP8_LINEARS for x in ("q", "s")]
+
+
 class VitWeightsDesc(ctypes.Structure):
     _fields_ = [("depth", c_int), ("out_dim", c_int), ("ln_eps", c_float), ("patch_order", c_int),
                 ("pe_w", c_void_p), ("pe_b", c_void_p), ("layers", ctypes.POINTER(VitLayerW)),
                 ("lnq_w", c_void_p), ("lnq_b", c_void_p), ("m0_w", c_void_p), ("m0_b", c_void_p),
                 ("m2_w", c_void_p), ("m2_b", c_void_p), ("window", c_int),
-                ("full_attention", ctypes.POINTER(ctypes.c_uint8))]
+                ("full_attention", ctypes.POINTER(ctypes.c_uint8)),
+                ("fp8_layers", ctypes.POINTER(VitLayerFp8))]
 
 # The Qwen2.5-VL tower's full-attention blocks (0-based) when windows are on
 QWEN25_FULL_BLOCKS = (7, 15, 23, 31)
@@ -65,6 +73,11 @@ _SIGS = {
     "vit_op_attention": (c_int, [c_void_p, c_int64, c_i32p, c_int, c_void_p, c_void_p, c_void_p]),
     "vit_op_wait_selftest": (c_int, [c_void_p, c_int64, c_void_p]),
     "vit_op_exp2_fma": (c_int, [c_void_p, c_void_p, c_int64, c_void_p]),
+    "vit_quantize_fp8": (c_int, [c_void_p, c_int64, c_int, c_void_p, c_void_p, c_void_p]),
+    "vit_op_gemm_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int, c_int,
+                                c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "vit_op_layernorm_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_float,
+                                     c_void_p]),
     "mrope_apply": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_int64, ctypes.c_double, c_i32p,
                             c_void_p]),
     "scatter_vision_tokens": (c_int, [c_void_p, c_int64, c_void_p, c_int64, c_int, c_void_p, c_int64, c_void_p,
@@ -171,13 +184,31 @@ def random_weights_device(depth: int, out_dim: int, seed: int, device="cuda", st
     return w
 
 
+def quantize_fp8(x: torch.Tensor, stream=None):
+    """E4M3 codes (uint8, same shape) and per-row power-of-two scales (fp32 [rows]) of a bf16
+    [rows, cols] device tensor, by vit_quantize_fp8."""
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.dim() == 2
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scales = torch.empty((x.shape[0],), dtype=torch.float32, device=x.device)
+    check(lib().vit_quantize_fp8(_ptr(x), x.shape[0], x.shape[1], _ptr(codes), _ptr(scales), _stream(stream)),
+          "vit_quantize_fp8")
+    return codes, scales
+
+
+def fp8_layers_device(weights: Dict, stream=None):
+    """Per layer {"qkv": (codes, scales), "proj": ..., "fc1": ..., "fc2": ...} of the device bf16
+    weights' four block linears, quantised on the device."""
+    return [{k: quantize_fp8(L[f"{k}_w"], stream) for k in FP8_LINEARS} for L in weights["layers"]]
+
+
 class VisionEncoder:
     """A validated weight view (vit_handle) and its workspace; ``encode`` runs vit_encode.
     window > 0 makes the windowed (Qwen2.5-VL) tower: blocks in ``full_blocks`` attend over the
-    whole frame, the others inside window x window patches."""
+    whole frame, the others inside window x window patches. fp8: per layer the E4M3 codes and
+    scales of the four block linears (``fp8_layers_device``): the fp8 tower."""
 
     def __init__(self, weights: Dict, out_dim: int, eps: float = 1e-6, patch_order: int = 0, window: int = 0,
-                 full_blocks: Sequence[int] = ()):
+                 full_blocks: Sequence[int] = (), fp8=None):
         self.weights = weights          # keeps the device tensors alive
         self.out_dim = out_dim
         depth = len(weights["layers"])
@@ -194,6 +225,14 @@ class VisionEncoder:
         d.window = int(window)
         self._full = (ctypes.c_uint8 * depth)(*[1 if l in set(full_blocks) else 0 for l in range(depth)])
         d.full_attention = ctypes.cast(self._full, ctypes.POINTER(ctypes.c_uint8))
+        self._fp8 = fp8                 # keeps the codes and scales alive
+        if fp8 is not None:
+            self._fp8_layers = (VitLayerFp8 * depth)()
+            for i, Lq in enumerate(fp8):
+                for k in FP8_LINEARS:
+                    setattr(self._fp8_layers[i], f"{k}_q", _ptr(Lq[k][0]))
+                    setattr(self._fp8_layers[i], f"{k}_s", _ptr(Lq[k][1]))
+            d.fp8_layers = self._fp8_layers
         self._desc = d
         h = c_void_p()
         check(lib().vit_weights_create(ctypes.byref(d), ctypes.byref(h)), "vit_weights_create")
@@ -306,6 +345,23 @@ def op_attention(qkv, cu_seqlens: Sequence[int], out, status=None, stream=None):
     check(lib().vit_op_attention(_ptr(qkv), qkv.shape[0], cu.ctypes.data_as(c_i32p), cu.shape[0] - 1, _ptr(out),
                                  _ptr(status), _stream(stream)), "vit_op_attention")
     return out
+
+
+def op_gemm_fp8(A, a_scale, B, b_scale, bias, C, epilogue, pos=None, rope_cs=None, status=None, stream=None):
+    M, K = A.shape
+    N = B.shape[0]
+    check(lib().vit_op_gemm_fp8(_ptr(A), _ptr(a_scale), _ptr(B), _ptr(b_scale), _ptr(bias), _ptr(C), M, N, K,
+                                epilogue, _ptr(pos), _ptr(rope_cs), _ptr(status), _stream(stream)), "vit_op_gemm_fp8")
+    return C
+
+
+def op_layernorm_fp8(X, gamma, beta, eps=1e-6, stream=None):
+    rows = X.shape[0]
+    codes = torch.empty((rows, syn.WIDTH), dtype=torch.uint8, device=X.device)
+    scales = torch.empty((rows,), dtype=torch.float32, device=X.device)
+    check(lib().vit_op_layernorm_fp8(_ptr(X), _ptr(gamma), _ptr(beta), _ptr(codes), _ptr(scales), rows, eps,
+                                     _stream(stream)), "vit_op_layernorm_fp8")
+    return codes, scales
 
 
 def op_exp2_fma(x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

@@ -1,7 +1,7 @@
 """Comparison helpers for the GPU-vs-oracle parity tests.
 
-Tolerances (derived in DESIGN.md, "Tolerances"). bf16 carries 8 significant bits, so one
-rounding to bf16 has relative error at most u = 2^-8 (the unit roundoff).
+Tolerances, derived from the arithmetic of the CUDA path. bf16 carries 8 significant bits, so
+one rounding to bf16 has relative error at most u = 2^-8 (the unit roundoff).
 * fp32 outputs of a bf16 x bf16 -> fp32 product: max|err| <= 1e-4 * max|ref| (fp32-accumulate path).
 * bf16 outputs: the fp32 result is rounded once to bf16, so |err| <= u * |ref| + 1e-4 * max|ref|.
 * attention: every weight of P is rounded to bf16 before P V (relative error <= u, weights sum to
