@@ -16,11 +16,9 @@
 //   warps 3..6  softmax of tile A, 7..10 of tile B, one query row per thread: scores from TMEM,
 //               online max / sum in fp32 with a lazy rescale (the exponent offset moves only when
 //               the running max, in log2 units, grows by more than 8), P in bf16 back to TMEM, O
-//               rescaled after the exponentials; the two warpgroups take turns at the MUFU
-//               (named barriers) so one group's loads and stores overlap the other's MUFU work,
-//               and a fixed share of every row's exponentials runs on the FMA pipe instead
-//               (exp2_fma2: range reduction + a minimax polynomial), computed before the
-//               group's MUFU turn, while the other group holds the MUFU; final O / l in bf16.
+//               rescaled after the exponentials; the two warpgroups take turns at the
+//               exponentials (named barriers) so one group's loads and stores overlap the
+//               other's MUFU work; final O / l written as bf16.
 // Work items are (segment, pair of query tiles), longest segments first; the work list travels
 // as a kernel parameter.
 #include <cuda_bf16.h>
@@ -48,15 +46,7 @@ constexpr int kMaxWorkPerLaunch = 4096;
 // Lazy rescaling: a row's exponent offset only moves when its running max grows by more than
 // this (log2 units), so P stays below 2^8 and O is rarely rescaled.
 constexpr float kRescaleThreshold = 8.0f;
-// Exponentials split between the two pipes: of every kFmaPeriod pairs of P columns, the first
-// kFmaPairs are computed on the FMA pipe (exp2_fma2), the others by the MUFU (ex2.approx). The
-// MUFU takes one warp instruction per 8 cycles on a sub-partition; one FMA-pipe exponential
-// costs about eight issue slots, so a small share balances the two.
-#ifndef VIT_ATTN_FMA_PAIRS
-#define VIT_ATTN_FMA_PAIRS 0
-#endif
-constexpr int kFmaPeriod = 8, kFmaPairs = VIT_ATTN_FMA_PAIRS;
-__host__ __device__ constexpr bool fma_pair(int i) { return (i % kFmaPeriod) < kFmaPairs; }
+
 // TMEM columns of query tile x: scores S_x (112), P_x (bf16 pairs, 56 used of 64), O_x (80).
 __host__ __device__ constexpr uint32_t col_s(int x) { return x * 112; }
 __host__ __device__ constexpr uint32_t col_p(int x) { return 224 + x * 64; }
@@ -72,6 +62,11 @@ struct AttnPlan {
     int work[kMaxWorkPerLaunch];      // (local segment << 16) | pair of query tiles
 };
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -245,13 +240,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int k = 0; k < kBKV; ++k)
                     if (k >= kv_valid) sr[k] = __float_as_uint(-INFINITY);
             }
+            // row max: eight independent chains of three-input maxima (max.f32 with three sources)
             float m8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) m8[i] = __uint_as_float(sr[i]);
 #pragma unroll
-            for (int k = 8; k < kBKV; k += 8)
+            for (int k = 8; k + 16 <= kBKV; k += 16)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], __uint_as_float(sr[k + i]));
+                for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], __uint_as_float(sr[k + i]), __uint_as_float(sr[k + 8 + i]));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], __uint_as_float(sr[kBKV - 8 + i]));
             const float mx =
                 fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
                 scale_log2;
@@ -264,31 +262,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float neg_m = -m_used;
             float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             uint32_t pk[56];
-            // the FMA-pipe share first, while the other group holds the MUFU
-#pragma unroll
-            for (int i = 0; i < kBKV / 2; ++i) {
-                if (!fma_pair(i)) continue;
-                float p0 = fmaf(__uint_as_float(sr[2 * i]), scale_log2, neg_m);
-                float p1 = fmaf(__uint_as_float(sr[2 * i + 1]), scale_log2, neg_m);
-                exp2_fma2(p0, p1);
-                r8[(i & 3) + 4 * ((i >> 2) & 1)] += p0 + p1;
-                pk[i] = pack_bf16x2(p0, p1);
-            }
-            named_bar_sync(my_turn, 256);                           // this group's MUFU turn
-            // groups of four pairs: up to eight independent exponentials in flight before their
-            // results are summed and packed, so the MUFU latency overlaps within one thread
+            named_bar_sync(my_turn, 256);                           // this group's turn
+            // groups of four pairs: eight independent exponentials in flight before their results
+            // are summed and packed, so the MUFU latency overlaps within one thread
 #pragma unroll
             for (int k = 0; k < kBKV; k += 8) {
                 float p[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if (!fma_pair((k + e) >> 1)) p[e] = fmaf(__uint_as_float(sr[k + e]), scale_log2, neg_m);
+                for (int e = 0; e < 8; ++e) p[e] = fmaf(__uint_as_float(sr[k + e]), scale_log2, neg_m);
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if (!fma_pair((k + e) >> 1)) p[e] = ex2(p[e]);
+                for (int e = 0; e < 8; ++e) p[e] = ex2(p[e]);
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
-                    if (fma_pair((k + e) >> 1)) continue;
                     r8[(e >> 1) + 4 * ((k >> 3) & 1)] += p[e] + p[e + 1];
                     pk[(k + e) >> 1] = pack_bf16x2(p[e], p[e + 1]);
                 }
