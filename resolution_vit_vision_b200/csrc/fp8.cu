@@ -49,8 +49,11 @@ __device__ __forceinline__ float warp_add(float v) {
 
 constexpr int kQWarps = 8;
 
-// One warp per row of `cols` bf16 values (cols a multiple of 8): max |x| in a first pass, the
-// codes in a second (the row is then in L1), eight values per lane per step.
+// One warp per row of `cols` bf16 values (cols a multiple of 8), eight values per lane per step.
+// CH > 0: the row is CH * 256 values wide and stays in registers between the max and the codes
+// (one read of the row); CH == 0: any width, the row is read twice (the second time mostly from
+// L1 or L2).
+template <int CH>
 __global__ void __launch_bounds__(kQWarps * 32)
     quantize_rows_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows, int cols, uint8_t *__restrict__ codes,
                          float *__restrict__ scales) {
@@ -58,8 +61,29 @@ __global__ void __launch_bounds__(kQWarps * 32)
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kQWarps + warp;
     if (row >= rows) return;
     const uint4 *src = reinterpret_cast<const uint4 *>(x + row * cols);
-    const int n8 = cols >> 3;
+    uint2 *dst = reinterpret_cast<uint2 *>(codes + row * cols);
     float amax = 0.f;
+    if (CH > 0) {
+        uint4 u[CH > 0 ? CH : 1];
+#pragma unroll
+        for (int i = 0; i < CH; ++i) u[i] = __ldcs(src + lane + 32 * i);
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+        }
+        const int e = fp8_scale_exp(warp_max(amax));
+        const float inv = exp2i(-e);
+#pragma unroll
+        for (int i = 0; i < CH; ++i)
+            dst[lane + 32 * i] =
+                make_uint2(e4m3x4(bf16_lo(u[i].x) * inv, bf16_hi(u[i].x) * inv, bf16_lo(u[i].y) * inv, bf16_hi(u[i].y) * inv),
+                           e4m3x4(bf16_lo(u[i].z) * inv, bf16_hi(u[i].z) * inv, bf16_lo(u[i].w) * inv, bf16_hi(u[i].w) * inv));
+        if (lane == 0) scales[row] = exp2i(e);
+        return;
+    }
+    const int n8 = cols >> 3;
     for (int c = lane; c < n8; c += 32) {
         const uint4 u = src[c];
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -68,7 +92,6 @@ __global__ void __launch_bounds__(kQWarps * 32)
     }
     const int e = fp8_scale_exp(warp_max(amax));
     const float inv = exp2i(-e);
-    uint2 *dst = reinterpret_cast<uint2 *>(codes + row * cols);
     for (int c = lane; c < n8; c += 32) {
         const uint4 u = src[c];
         dst[c] = make_uint2(e4m3x4(bf16_lo(u.x) * inv, bf16_hi(u.x) * inv, bf16_lo(u.y) * inv, bf16_hi(u.y) * inv),
@@ -136,8 +159,13 @@ namespace vith {
 int quantize_rows_launch(const void *x, int64_t rows, int cols, void *codes, float *scales, cudaStream_t s) {
     if (rows <= 0) return VIT_OK;
     const int64_t blocks = (rows + vitk::kQWarps - 1) / vitk::kQWarps;
-    vitk::quantize_rows_kernel<<<static_cast<unsigned>(blocks), vitk::kQWarps * 32, 0, s>>>(
-        static_cast<const __nv_bfloat16 *>(x), rows, cols, static_cast<uint8_t *>(codes), scales);
+    const auto *xb = static_cast<const __nv_bfloat16 *>(x);
+    auto *cb = static_cast<uint8_t *>(codes);
+    const dim3 grid(static_cast<unsigned>(blocks)), block(vitk::kQWarps * 32);
+    // the widths of the tower's product inputs keep their rows in registers (one read)
+    if (cols == VIT_MLP) vitk::quantize_rows_kernel<VIT_MLP / 256><<<grid, block, 0, s>>>(xb, rows, cols, cb, scales);
+    else if (cols == VIT_WIDTH) vitk::quantize_rows_kernel<VIT_WIDTH / 256><<<grid, block, 0, s>>>(xb, rows, cols, cb, scales);
+    else vitk::quantize_rows_kernel<0><<<grid, block, 0, s>>>(xb, rows, cols, cb, scales);
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 
