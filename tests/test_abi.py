@@ -129,3 +129,62 @@ def test_decoder_steps_reject_bad_arguments_before_cuda(lib):
     assert lib.scatter_vision_tokens(p, (1 << 18) + 1, p, 100, 64, p, 2, p, None, None) == nv.VIT_ERR_ARG
     assert lib.scatter_vision_tokens(p, 10, p, 100, 64, None, 2, p, None, None) == nv.VIT_ERR_ARG
     assert lib.scatter_vision_tokens(p, 10, ctypes.c_void_p(0x10004), 100, 64, p, 2, p, None, None) == nv.VIT_ERR_ALIGN
+
+
+def test_fp8_entry_points_reject_bad_arguments_before_cuda(lib):
+    from resolution_vit_vision_b200 import native as nv
+    p = ctypes.c_void_p(0x10000)
+    # vit_quantize_fp8: width a multiple of 8 in 8..65536, pointers present and 16-byte aligned
+    assert lib.vit_quantize_fp8(p, 4, 12, p, p, None) == nv.VIT_ERR_ARG
+    assert lib.vit_quantize_fp8(p, 4, 65544, p, p, None) == nv.VIT_ERR_ARG
+    assert lib.vit_quantize_fp8(None, 4, 64, p, p, None) == nv.VIT_ERR_ARG
+    assert lib.vit_quantize_fp8(p, -1, 64, p, p, None) == nv.VIT_ERR_ARG
+    assert lib.vit_quantize_fp8(ctypes.c_void_p(0x10008), 4, 64, p, p, None) == nv.VIT_ERR_ALIGN
+    assert lib.vit_quantize_fp8(p, 0, 64, None, None, None) == nv.VIT_OK       # nothing to do
+    # vit_op_gemm_fp8: scales required, K a multiple of 16, QKV_ROPE only for N = 3840
+    args = dict(A=p, sa=p, B=p, sb=p, bias=None, C=p, M=64, N=256, K=128, epi=nv.EPI_ADD_F32)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.vit_op_gemm_fp8(a["A"], a["sa"], a["B"], a["sb"], a["bias"], a["C"], a["M"], a["N"], a["K"],
+                                   a["epi"], None, None, None, None)
+    assert call(sa=None) == nv.VIT_ERR_ARG
+    assert call(sb=None) == nv.VIT_ERR_ARG
+    assert call(K=120) == nv.VIT_ERR_ARG
+    assert call(N=250) == nv.VIT_ERR_ARG
+    assert call(epi=nv.EPI_QKV_ROPE) == nv.VIT_ERR_ARG
+    assert call(epi=9) == nv.VIT_ERR_ARG
+    assert call(sb=ctypes.c_void_p(0x10004)) == nv.VIT_ERR_ALIGN
+    assert call(M=(1 << 30) + 1) == nv.VIT_ERR_LIMIT
+    # vit_op_layernorm_fp8
+    assert lib.vit_op_layernorm_fp8(p, p, None, p, None, 4, 1e-6, None) == nv.VIT_ERR_ARG
+    assert lib.vit_op_layernorm_fp8(p, p, None, p, p, 4, 0.0, None) == nv.VIT_ERR_ARG
+    assert lib.vit_op_layernorm_fp8(ctypes.c_void_p(0x10008), p, None, p, p, 4, 1e-6, None) == nv.VIT_ERR_ALIGN
+    # vit_op_exp2_fma
+    assert lib.vit_op_exp2_fma(None, p, 4, None) == nv.VIT_ERR_ARG
+    assert lib.vit_op_exp2_fma(p, p, -1, None) == nv.VIT_ERR_ARG
+    assert lib.vit_op_exp2_fma(None, None, 0, None) == nv.VIT_OK
+
+
+def test_weights_create_validates_fp8_layers_before_cuda(lib):
+    # an fp8 descriptor with a missing code pointer is refused before any device call
+    from resolution_vit_vision_b200 import native as nv
+    p = 0x10000
+    layers = (nv.VitLayerW * 1)()
+    for k in ("ln1_w", "ln2_w"):
+        setattr(layers[0], k, p)
+    q8 = (nv.VitLayerFp8 * 1)()
+    for f, _ in nv.VitLayerFp8._fields_:
+        setattr(q8[0], f, p)
+    d = nv.VitWeightsDesc()
+    d.depth, d.out_dim, d.ln_eps, d.patch_order = 1, 1536, 1e-6, 0
+    d.pe_w = d.lnq_w = d.m0_w = d.m2_w = p
+    d.layers = layers
+    d.fp8_layers = q8
+    h = ctypes.c_void_p()
+    q8[0].fc2_q = None
+    assert lib.vit_weights_create(ctypes.byref(d), ctypes.byref(h)) == nv.VIT_ERR_ARG
+    q8[0].fc2_q = p + 8
+    assert lib.vit_weights_create(ctypes.byref(d), ctypes.byref(h)) == nv.VIT_ERR_ALIGN
+    d.fp8_layers = None                                  # bf16 tower: the linears are then required
+    assert lib.vit_weights_create(ctypes.byref(d), ctypes.byref(h)) == nv.VIT_ERR_ARG
