@@ -206,6 +206,7 @@ int ensure_workspace(vit_handle *h, int64_t P) {
 int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n_images, int64_t P, void *out,
                   cudaStream_t s) {
     const vit_weights_desc &d = h->desc;
+    auto nw = vith::gemm_use_narrow;   // which prebuilt weight map (256 x 256 or 256 x 128 tiles) a product takes
     if (h->prof && h->ev_used) prof_collect(h);
     h->last_stream = s;
     int64_t &nl = h->launches;
@@ -272,7 +273,8 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
 
     {
         ProfScope ps(h, s, P_PE);
-        VIT_TRY(vith::gemm_launch(mPatch, h->pe_map, cX, d.pe_b, P, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32,
+        VIT_TRY(vith::gemm_launch(mPatch, nw(P, VIT_WIDTH, VIT_EPI_STORE_F32) ? h->pe_map_n : h->pe_map, cX, d.pe_b, P,
+                                  VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32,
                                   nullptr, nullptr, h->status, s));
         ++nl;
     }
@@ -313,7 +315,8 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
         }
         {
             ProfScope ps(h, s, P_PROJ);
-            VIT_TRY(vith::gemm_launch(f8 ? mQ8w : mH, lm.proj, cX, L.proj_b, P, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32,
+            VIT_TRY(vith::gemm_launch(f8 ? mQ8w : mH, nw(P, VIT_WIDTH, VIT_EPI_ADD_F32) ? lm.proj_n : lm.proj, cX,
+                                      L.proj_b, P, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32,
                                       nullptr, nullptr, h->status, s, f8 ? h->S8 : nullptr,
                                       f8 ? L8->proj_s : nullptr));
             ++nl;
@@ -326,7 +329,8 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
         }
         {
             ProfScope ps(h, s, P_FC1);
-            VIT_TRY(vith::gemm_launch(f8 ? mQ8w : mH, lm.fc1, cF, L.fc1_b, P, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16,
+            VIT_TRY(vith::gemm_launch(f8 ? mQ8w : mH, nw(P, VIT_MLP, VIT_EPI_GELU_BF16) ? lm.fc1_n : lm.fc1, cF,
+                                      L.fc1_b, P, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16,
                                       nullptr, nullptr, h->status, s, f8 ? h->S8 : nullptr,
                                       f8 ? L8->fc1_s : nullptr));
             ++nl;
@@ -338,7 +342,8 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
         }
         {
             ProfScope ps(h, s, P_FC2);
-            VIT_TRY(vith::gemm_launch(f8 ? mQ8m : mF, lm.fc2, cX, L.fc2_b, P, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32,
+            VIT_TRY(vith::gemm_launch(f8 ? mQ8m : mF, nw(P, VIT_WIDTH, VIT_EPI_ADD_F32) ? lm.fc2_n : lm.fc2, cX,
+                                      L.fc2_b, P, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32,
                                       nullptr, nullptr, h->status, s, f8 ? h->S8 : nullptr,
                                       f8 ? L8->fc2_s : nullptr));
             ++nl;
@@ -352,13 +357,15 @@ int encode_device(vit_handle *h, const void *patches, const int32_t *grid, int n
     }
     {
         ProfScope ps(h, s, P_M0);
-        VIT_TRY(vith::gemm_launch(mH4, h->m0_map, cF4, d.m0_b, M4, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16,
+        VIT_TRY(vith::gemm_launch(mH4, nw(M4, VIT_MERGE_DIM, VIT_EPI_GELU_BF16) ? h->m0_map_n : h->m0_map, cF4, d.m0_b,
+                                  M4, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16,
                                   nullptr, nullptr, h->status, s));
         ++nl;
     }
     {
         ProfScope ps(h, s, P_M2);
-        VIT_TRY(vith::gemm_launch(mF4, h->m2_map, cOut, d.m2_b, M4, d.out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16,
+        VIT_TRY(vith::gemm_launch(mF4, nw(M4, d.out_dim, VIT_EPI_STORE_BF16) ? h->m2_map_n : h->m2_map, cOut, d.m2_b,
+                                  M4, d.out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16,
                                   nullptr, nullptr, h->status, s));
         ++nl;
     }
@@ -520,6 +527,12 @@ int vit_weights_create(const vit_weights_desc *d, vit_handle **out) {
     rc = vith::gemm_make_b_map(&h->pe_map, d->pe_w, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32);
     if (rc == VIT_OK) rc = vith::gemm_make_b_map(&h->m0_map, d->m0_w, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16);
     if (rc == VIT_OK) rc = vith::gemm_make_b_map(&h->m2_map, d->m2_w, d->out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16);
+    if (rc == VIT_OK)
+        rc = vith::gemm_make_b_map(&h->pe_map_n, d->pe_w, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32, false, true);
+    if (rc == VIT_OK)
+        rc = vith::gemm_make_b_map(&h->m0_map_n, d->m0_w, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16, false, true);
+    if (rc == VIT_OK)
+        rc = vith::gemm_make_b_map(&h->m2_map_n, d->m2_w, d->out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16, false, true);
     for (int l = 0; l < d->depth && rc == VIT_OK; ++l) {
         const vit_layer_w &L = h->layers[l];
         vith::LayerMaps &m = h->maps[l];
@@ -532,6 +545,15 @@ int vit_weights_create(const vit_weights_desc *d, vit_handle **out) {
             rc = vith::gemm_make_b_map(&m.fc1, f8 ? Q->fc1_q : L.fc1_w, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16, f8);
         if (rc == VIT_OK)
             rc = vith::gemm_make_b_map(&m.fc2, f8 ? Q->fc2_q : L.fc2_w, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32, f8);
+        if (rc == VIT_OK)
+            rc = vith::gemm_make_b_map(&m.proj_n, f8 ? Q->proj_q : L.proj_w, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32, f8,
+                                       true);
+        if (rc == VIT_OK)
+            rc = vith::gemm_make_b_map(&m.fc1_n, f8 ? Q->fc1_q : L.fc1_w, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16, f8,
+                                       true);
+        if (rc == VIT_OK)
+            rc = vith::gemm_make_b_map(&m.fc2_n, f8 ? Q->fc2_q : L.fc2_w, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32, f8,
+                                       true);
     }
     if (rc != VIT_OK) return rc;
     *out = h.release();
@@ -656,7 +678,7 @@ int vit_op_gemm(const void *A, const void *B, const void *bias, void *C, int64_t
     if (!aligned16(A) || !aligned16(B) || !aligned16(C) || (bias && !aligned16(bias))) return VIT_ERR_ALIGN;
     CUtensorMap ta, tb, tc;
     int rc = vith::gemm_make_a_map(&ta, A, M, K);
-    if (rc == VIT_OK) rc = vith::gemm_make_b_map(&tb, B, N, K, epilogue);
+    if (rc == VIT_OK) rc = vith::gemm_make_b_map(&tb, B, N, K, epilogue, false, vith::gemm_use_narrow(M, N, epilogue));
     if (rc == VIT_OK) rc = vith::gemm_make_c_map(&tc, C, M, N, epilogue);
     if (rc != VIT_OK) return rc;
     return vith::gemm_launch(ta, tb, tc, bias, M, N, K, epilogue, pos, rope_cs, dev_status,
@@ -675,7 +697,7 @@ int vit_op_gemm_fp8(const void *A, const float *a_scale, const void *B, const fl
         return VIT_ERR_ALIGN;
     CUtensorMap ta, tb, tc;
     int rc = vith::gemm_make_a_map(&ta, A, M, K, true);
-    if (rc == VIT_OK) rc = vith::gemm_make_b_map(&tb, B, N, K, epilogue, true);
+    if (rc == VIT_OK) rc = vith::gemm_make_b_map(&tb, B, N, K, epilogue, true, vith::gemm_use_narrow(M, N, epilogue));
     if (rc == VIT_OK) rc = vith::gemm_make_c_map(&tc, C, M, N, epilogue);
     if (rc != VIT_OK) return rc;
     return vith::gemm_launch(ta, tb, tc, bias, M, N, K, epilogue, pos, rope_cs, dev_status,

@@ -38,7 +38,7 @@ constexpr int kEpiBarrier = 1;    // named barrier of the 128 epilogue threads
 
 template <int BN>
 struct GemmShape {
-    static constexpr int STAGES = BN == 240 ? 5 : 6;
+    static constexpr int STAGES = BN == 240 ? 5 : (BN == 128 ? 8 : 6);
     static constexpr int A_BYTES = kBM * kBK * 2;
     static constexpr int B_BYTES = (BN / 2) * kBK * 2;   // this CTA's half of the B tile
     static constexpr int ACC_STRIDE = 256;    // TMEM columns between the two accumulators
@@ -420,8 +420,16 @@ int gemm_make_a_map(CUtensorMap *map, const void *A, int64_t M, int K, bool f8) 
                    vitk::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue, bool f8) {
-    const uint32_t bn = (epilogue == VIT_EPI_QKV_ROPE) ? 240 : 256;   // each CTA of a pair loads half
+// Narrow tiles (256 x 128) when the 256 x 256 tiles of a product would not fill the device's SM
+// pairs once (a single small image: M = 1024 gives 20 tiles of N = 1280 for 74 pairs).
+bool gemm_use_narrow(int64_t M, int N, int epilogue) {
+    if (epilogue == VIT_EPI_QKV_ROPE) return false;   // the rope epilogue needs whole 80-wide heads
+    const int64_t tiles = ((M + 2 * vitk::kBM - 1) / (2 * vitk::kBM)) * ((N + 255) / 256);
+    return tiles < device_sm_count() / 2;
+}
+
+int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue, bool f8, bool narrow) {
+    const uint32_t bn = (epilogue == VIT_EPI_QKV_ROPE) ? 240 : (narrow ? 128 : 256);   // each CTA of a pair loads half
     if (f8)
         return tmap_2d(map, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, static_cast<uint64_t>(K), 2 * vitk::kBK,
                        bn / 2, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -504,6 +512,25 @@ int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap 
     p.m_tiles = static_cast<int>((M + 2 * vitk::kBM - 1) / (2 * vitk::kBM));
     const int kblk = f8 ? 2 * vitk::kBK : vitk::kBK;   // elements per 128-byte k-block
     p.k_blocks = (K + kblk - 1) / kblk;
+    if (gemm_use_narrow(M, N, epilogue)) {   // the B map was made with narrow = true
+        p.n_tiles = (N + 127) / 128;
+        switch (epilogue) {
+            case VIT_EPI_STORE_F32:
+                return f8 ? launch_one<128, VIT_EPI_STORE_F32, true>(ta, tb, tc, p, s)
+                          : launch_one<128, VIT_EPI_STORE_F32, false>(ta, tb, tc, p, s);
+            case VIT_EPI_ADD_F32:
+                return f8 ? launch_one<128, VIT_EPI_ADD_F32, true>(ta, tb, tc, p, s)
+                          : launch_one<128, VIT_EPI_ADD_F32, false>(ta, tb, tc, p, s);
+            case VIT_EPI_STORE_BF16:
+                return f8 ? launch_one<128, VIT_EPI_STORE_BF16, true>(ta, tb, tc, p, s)
+                          : launch_one<128, VIT_EPI_STORE_BF16, false>(ta, tb, tc, p, s);
+            case VIT_EPI_GELU_BF16:
+                return f8 ? launch_one<128, VIT_EPI_GELU_BF16, true>(ta, tb, tc, p, s)
+                          : launch_one<128, VIT_EPI_GELU_BF16, false>(ta, tb, tc, p, s);
+            default:
+                return VIT_ERR_ARG;
+        }
+    }
     switch (epilogue) {
         case VIT_EPI_QKV_ROPE:
             p.n_tiles = N / 240;

@@ -12,6 +12,7 @@
 namespace vith {
 struct LayerMaps {
     CUtensorMap qkv, proj, fc1, fc2;
+    CUtensorMap proj_n, fc1_n, fc2_n;   // the same weights for 256 x 128 tiles (small batches)
 };
 constexpr int kProfClasses = 12;
 }  // namespace vith
@@ -23,6 +24,7 @@ struct vit_handle {
     std::vector<vit_layer_fp8> fp8;        // [depth] when the block linears run in E4M3, else empty
     std::vector<vith::LayerMaps> maps;     // of the bf16 weights, or of the E4M3 codes
     CUtensorMap pe_map{}, m0_map{}, m2_map{};
+    CUtensorMap pe_map_n{}, m0_map_n{}, m2_map_n{};   // for 256 x 128 tiles
     int device = 0;
 
     // workspace

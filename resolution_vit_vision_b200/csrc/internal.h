@@ -23,9 +23,13 @@ int check_device();   // VIT_OK when the current device is sm_100
 // ---- GEMM (gemm.cu). A bf16 [M, K], B bf16 [N, K]. The B map may be prebuilt (weights).
 // f8: E4M3 codes (one byte per element) instead of bf16
 int gemm_make_a_map(CUtensorMap *map, const void *A, int64_t M, int K, bool f8 = false);
-int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue, bool f8 = false);
+// narrow: the map of 256 x 128 tiles, which gemm_launch uses when gemm_use_narrow(M, N, epilogue)
+int gemm_make_b_map(CUtensorMap *map, const void *B, int N, int K, int epilogue, bool f8 = false,
+                    bool narrow = false);
+bool gemm_use_narrow(int64_t M, int N, int epilogue);
 // C [M, N]: fp32 for STORE_F32 / ADD_F32 (the output is written, or added, by TMA), else bf16
 int gemm_make_c_map(CUtensorMap *map, void *C, int64_t M, int N, int epilogue);
+// The B map must be made with narrow = gemm_use_narrow(M, N, epilogue).
 // a_scale != NULL selects the E4M3 product: A and B are codes (maps made with f8), a_scale [M] and
 // b_scale [N] their per-row power-of-two scales, applied to the accumulator before the bias
 int gemm_launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc, const void *bias, int64_t M,

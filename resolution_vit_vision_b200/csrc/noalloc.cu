@@ -104,6 +104,7 @@ extern "C" int vit_encode_noalloc(const void *patches, const int32_t *grid_thw, 
         for (int t = 0; t < grid_thw[3 * i]; ++t, ++n_seg) cu[n_seg + 1] = cu[n_seg] + grid_thw[3 * i + 1] * grid_thw[3 * i + 2];
     const int64_t M4 = P / 4;
     const vit_weights_desc &d = h->desc;
+    auto nw = vith::gemm_use_narrow;   // the weight map matching the tile width gemm_launch picks
 
     NA_TRY(vith::positions_launch_stack(grid_thw, n_images, P, d.patch_order, pos, merge_row, s));
     CUtensorMap mPatch, mH, mF, mH4, mF4;
@@ -120,7 +121,7 @@ extern "C" int vit_encode_noalloc(const void *patches, const int32_t *grid_thw, 
     NA_TRY(vith::gemm_make_c_map(&cF, F, P, VIT_MLP, VIT_EPI_GELU_BF16));
     NA_TRY(vith::gemm_make_c_map(&cF4, F, M4, VIT_MERGE_DIM, VIT_EPI_GELU_BF16));
     NA_TRY(vith::gemm_make_c_map(&cOut, out, M4, d.out_dim, VIT_EPI_STORE_BF16));
-    NA_TRY(vith::gemm_launch(mPatch, h->pe_map, cX, d.pe_b, P, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32, nullptr,
+    NA_TRY(vith::gemm_launch(mPatch, nw(P, VIT_WIDTH, VIT_EPI_STORE_F32) ? h->pe_map_n : h->pe_map, cX, d.pe_b, P, VIT_WIDTH, VIT_PATCH_DIM, VIT_EPI_STORE_F32, nullptr,
                              nullptr, dev_status, s));
     for (int l = 0; l < d.depth; ++l) {
         const vit_layer_w &L = h->layers[l];
@@ -129,19 +130,19 @@ extern "C" int vit_encode_noalloc(const void *patches, const int32_t *grid_thw, 
         NA_TRY(vith::gemm_launch(mH, lm.qkv, cQKV, L.qkv_b, P, 3 * VIT_WIDTH, VIT_WIDTH, VIT_EPI_QKV_ROPE, pos,
                                  rope_cs, dev_status, s));
         NA_TRY(vith::attn_launch_stack(mQKV, cu, n_seg, H, dev_status, s));
-        NA_TRY(vith::gemm_launch(mH, lm.proj, cX, L.proj_b, P, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32, nullptr, nullptr,
+        NA_TRY(vith::gemm_launch(mH, nw(P, VIT_WIDTH, VIT_EPI_ADD_F32) ? lm.proj_n : lm.proj, cX, L.proj_b, P, VIT_WIDTH, VIT_WIDTH, VIT_EPI_ADD_F32, nullptr, nullptr,
                                  dev_status, s));
         NA_TRY(vith::layernorm_launch(X, L.ln2_w, L.ln2_b, H, P, d.ln_eps, nullptr, s));
-        NA_TRY(vith::gemm_launch(mH, lm.fc1, cF, L.fc1_b, P, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16, nullptr, nullptr,
+        NA_TRY(vith::gemm_launch(mH, nw(P, VIT_MLP, VIT_EPI_GELU_BF16) ? lm.fc1_n : lm.fc1, cF, L.fc1_b, P, VIT_MLP, VIT_WIDTH, VIT_EPI_GELU_BF16, nullptr, nullptr,
                                  dev_status, s));
-        NA_TRY(vith::gemm_launch(mF, lm.fc2, cX, L.fc2_b, P, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32, nullptr, nullptr,
+        NA_TRY(vith::gemm_launch(mF, nw(P, VIT_WIDTH, VIT_EPI_ADD_F32) ? lm.fc2_n : lm.fc2, cX, L.fc2_b, P, VIT_WIDTH, VIT_MLP, VIT_EPI_ADD_F32, nullptr, nullptr,
                                  dev_status, s));
         h->launches += 7;
     }
     NA_TRY(vith::layernorm_launch(X, d.lnq_w, d.lnq_b, H, P, d.ln_eps, d.patch_order == 1 ? merge_row : nullptr, s));
-    NA_TRY(vith::gemm_launch(mH4, h->m0_map, cF4, d.m0_b, M4, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16, nullptr,
+    NA_TRY(vith::gemm_launch(mH4, nw(M4, VIT_MERGE_DIM, VIT_EPI_GELU_BF16) ? h->m0_map_n : h->m0_map, cF4, d.m0_b, M4, VIT_MERGE_DIM, VIT_MERGE_DIM, VIT_EPI_GELU_BF16, nullptr,
                              nullptr, dev_status, s));
-    NA_TRY(vith::gemm_launch(mF4, h->m2_map, cOut, d.m2_b, M4, d.out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16, nullptr,
+    NA_TRY(vith::gemm_launch(mF4, nw(M4, d.out_dim, VIT_EPI_STORE_BF16) ? h->m2_map_n : h->m2_map, cOut, d.m2_b, M4, d.out_dim, VIT_MERGE_DIM, VIT_EPI_STORE_BF16, nullptr,
                              nullptr, dev_status, s));
     h->launches += 5;
     return VIT_OK;

@@ -24,6 +24,8 @@ def _status():
 
 
 # ------------------------------------------------------------------ GEMM
+# Products with fewer 256 x 256 tiles than the device has SM pairs run on 256 x 128 tiles
+# (gemm_use_narrow); the first seven cases take that path, the last two the wide one.
 GEMM_CASES = [
     # (M, N, K): ragged M over several tiles, K tail (1176 = 18*64 + 24), N tails (N % 256 != 0)
     (300, 1280, 1176),
@@ -33,6 +35,8 @@ GEMM_CASES = [
     (385, 1280, 5120),
     (1, 3584, 5120),
     (200, 304, 72),
+    (4800, 1280, 1280),      # enough 256 x 256 tiles to fill the SM pairs: the wide tiles
+    (2100, 5120, 1280),
 ]
 
 
