@@ -72,15 +72,17 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def ncu_traffic(kernel_class):
+def ncu_traffic(kernel_class, workload):
     """DRAM bytes per launch from the committed ncu capture, or None when the kernel's source has
-    changed since the counters were taken."""
+    changed since the counters were taken or the capture was of another workload."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         rec = json.load(open(p))[kernel_class]
         src = open(os.path.join(ROOT, rec["source"]), "rb").read()
     except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("workload", "mixed8") != workload:
         return None
     return rec["bytes_per_launch"] if hashlib.sha1(src).hexdigest() == rec["sha1"] else None
 
@@ -576,7 +578,8 @@ def main():
               key=lambda n: kernels[n]["ms_per_step"])
     top_peak = 2.0 * tc_peak if top in f8_classes else tc_peak
     roof = {"kernel": top, "bound": "tensor", "achieved": kernels[top]["tflops"], "peak": top_peak,
-            "unit": "TFLOP/s", "frac": kernels[top]["frac"], "traffic": None if args.fp8 else ncu_traffic(top),
+            "unit": "TFLOP/s", "frac": kernels[top]["frac"],
+            "traffic": None if (args.fp8 or args.window) else ncu_traffic(top, wl.name),
             "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside the step)" +
                            (" x 2 (nominal fp8 / bf16 ratio)" if top in f8_classes else "")}
 
