@@ -124,6 +124,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
+    // the previous kernel of the stream (the QKV product) has completed from here on; tensor
+    // memory is taken only after it
+    pdl_wait();
+    pdl_trigger();
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
@@ -402,9 +406,11 @@ int launch_plans(vitk::AttnPlan &plan, const int *order, int n_seg,
     plan.n_work = 0;
     auto flush = [&]() {
         if (plan.n_work > 0) {
-            vitk::attn_tc_kernel<<<plan.n_work * VIT_HEADS, vitk::kAttnThreads, vitk::kAttnSmem, s>>>(
-                tqkv.q, tqkv.kv, plan, static_cast<__nv_bfloat16 *>(out), status);
-            if (cudaGetLastError() != cudaSuccess) return false;
+            if (launch_pdl(vitk::attn_tc_kernel, dim3(plan.n_work * VIT_HEADS), dim3(vitk::kAttnThreads),
+                           vitk::kAttnSmem, s, 1, tqkv.q, tqkv.kv, plan, static_cast<__nv_bfloat16 *>(out),
+                           status) != cudaSuccess ||
+                cudaGetLastError() != cudaSuccess)
+                return false;
         }
         plan.n_seg = 0;
         plan.n_work = 0;

@@ -57,6 +57,8 @@ template <int CH>
 __global__ void __launch_bounds__(kQWarps * 32)
     quantize_rows_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows, int cols, uint8_t *__restrict__ codes,
                          float *__restrict__ scales) {
+    pdl_wait();                                   // the rows are the previous kernel's output
+    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kQWarps + warp;
     if (row >= rows) return;
@@ -107,6 +109,8 @@ __global__ void __launch_bounds__(kLnWarps8 * 32)
     layernorm_fp8_kernel(const float *__restrict__ X, const __nv_bfloat16 *__restrict__ gamma,
                          const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ codes,
                          float *__restrict__ scales, int64_t rows, float eps) {
+    pdl_wait();
+    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kLnWarps8 + warp;
     if (row >= rows) return;
@@ -163,9 +167,10 @@ int quantize_rows_launch(const void *x, int64_t rows, int cols, void *codes, flo
     auto *cb = static_cast<uint8_t *>(codes);
     const dim3 grid(static_cast<unsigned>(blocks)), block(vitk::kQWarps * 32);
     // the widths of the tower's product inputs keep their rows in registers (one read)
-    if (cols == VIT_MLP) vitk::quantize_rows_kernel<VIT_MLP / 256><<<grid, block, 0, s>>>(xb, rows, cols, cb, scales);
-    else if (cols == VIT_WIDTH) vitk::quantize_rows_kernel<VIT_WIDTH / 256><<<grid, block, 0, s>>>(xb, rows, cols, cb, scales);
-    else vitk::quantize_rows_kernel<0><<<grid, block, 0, s>>>(xb, rows, cols, cb, scales);
+    auto *k = cols == VIT_MLP     ? vitk::quantize_rows_kernel<VIT_MLP / 256>
+              : cols == VIT_WIDTH ? vitk::quantize_rows_kernel<VIT_WIDTH / 256>
+                                  : vitk::quantize_rows_kernel<0>;
+    if (launch_pdl(k, grid, block, 0, s, 1, xb, rows, cols, cb, scales) != cudaSuccess) return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 
@@ -173,9 +178,10 @@ int layernorm_fp8_launch(const float *X, const void *gamma, const void *beta, vo
                          int64_t rows, float eps, cudaStream_t s) {
     if (rows <= 0) return VIT_OK;
     const int64_t blocks = (rows + vitk::kLnWarps8 - 1) / vitk::kLnWarps8;
-    vitk::layernorm_fp8_kernel<<<static_cast<unsigned>(blocks), vitk::kLnWarps8 * 32, 0, s>>>(
-        X, static_cast<const __nv_bfloat16 *>(gamma), static_cast<const __nv_bfloat16 *>(beta),
-        static_cast<uint8_t *>(codes), scales, rows, eps);
+    if (launch_pdl(vitk::layernorm_fp8_kernel, dim3(static_cast<unsigned>(blocks)), dim3(vitk::kLnWarps8 * 32), 0, s,
+                   1, X, static_cast<const __nv_bfloat16 *>(gamma), static_cast<const __nv_bfloat16 *>(beta),
+                   static_cast<uint8_t *>(codes), scales, rows, eps) != cudaSuccess)
+        return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 

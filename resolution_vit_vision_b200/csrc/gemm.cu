@@ -192,6 +192,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
+    // The previous kernel of the stream has completed from here on (the operands are its output);
+    // tensor memory is taken only after it, so no CTA holds any while it waits.
+    pdl_wait();
+    pdl_trigger();
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
         tmem_relinquish_pair();
@@ -466,18 +470,18 @@ static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtens
         if (dev < 64) configured[dev] = true;
     }
     static int max_clusters[64] = {};   // pairs that fit on the device at once (set with the attribute)
-    cudaLaunchConfig_t cfg{};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(vitk::kGemmThreads);
-    cfg.dynamicSmemBytes = S::SMEM;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     if (dev < 64 && max_clusters[dev] == 0) {
+        cudaLaunchConfig_t cfg{};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.blockDim = dim3(vitk::kGemmThreads);
+        cfg.dynamicSmemBytes = S::SMEM;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
         cfg.gridDim = dim3(2 * 74);
         int n = 0;
         if (cudaOccupancyMaxActiveClusters(&n, vitk::gemm_tc_kernel<BN, EPI, F8>, &cfg) != cudaSuccess || n < 1) {
@@ -488,8 +492,10 @@ static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtens
     }
     const int total = p.m_tiles * p.n_tiles;
     const int pairs = dev < 64 ? max_clusters[dev] : device_sm_count() / 2;
-    cfg.gridDim = dim3(2 * (total < pairs ? total : pairs));
-    if (cudaLaunchKernelEx(&cfg, vitk::gemm_tc_kernel<BN, EPI, F8>, ta, tb, tc, p) != cudaSuccess) return VIT_ERR_CUDA;
+    const dim3 grid(2 * (total < pairs ? total : pairs));
+    if (launch_pdl(vitk::gemm_tc_kernel<BN, EPI, F8>, grid, dim3(vitk::kGemmThreads), S::SMEM, s, 2, ta, tb, tc, p) !=
+        cudaSuccess)
+        return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 

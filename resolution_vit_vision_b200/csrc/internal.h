@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <utility>
 #include <vector>
 
 #include "../../include/vit.h"
@@ -11,6 +12,29 @@
 #include "../../include/vit_ops.h"
 
 namespace vith {
+
+// Launches kernel k with programmatic stream serialisation: k may start while the previous kernel
+// of stream s finishes, so every such kernel calls pdl_wait() (ptx.cuh) before it touches global
+// memory. cluster_x > 1 also launches it in clusters of that many CTAs.
+template <typename... P, typename... A>
+inline cudaError_t launch_pdl(void (*k)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster_x,
+                              A &&...args) {
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = cluster_x > 1 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, k, std::forward<A>(args)...);
+}
 
 // ---- tensor maps (driver entry point fetched through the runtime, no -lcuda needed)
 int tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes, uint64_t inner,

@@ -28,6 +28,8 @@ __global__ void __launch_bounds__(kLnWarps * 32)
     layernorm_kernel(const float *__restrict__ X, const __nv_bfloat16 *__restrict__ gamma,
                      const __nv_bfloat16 *__restrict__ beta, __nv_bfloat16 *__restrict__ Y, int64_t rows, float eps,
                      const int32_t *__restrict__ out_row) {
+    pdl_wait();                                   // the rows are the previous kernel's output
+    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kLnWarps + warp;
     if (row >= rows) return;
@@ -92,6 +94,8 @@ struct ImageTable {
 // merge_row[r]: the row patch r takes in block order (the merger reads four consecutive rows).
 __global__ void positions_kernel(const __grid_constant__ ImageTable tab, int64_t P, int patch_order,
                                  int32_t *__restrict__ pos, int32_t *__restrict__ merge_row) {
+    pdl_wait();                                   // the previous encode may still read pos / merge_row
+    pdl_trigger();
     const int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (r >= P) return;
     int lo = 0, hi = tab.n - 1;   // last image with row_start <= r
@@ -288,9 +292,10 @@ int layernorm_launch(const float *X, const void *gamma, const void *beta, void *
                      const int32_t *out_row, cudaStream_t s) {
     if (rows <= 0) return VIT_OK;
     const int64_t blocks = (rows + vitk::kLnWarps - 1) / vitk::kLnWarps;
-    vitk::layernorm_kernel<<<static_cast<unsigned>(blocks), vitk::kLnWarps * 32, 0, s>>>(
-        X, static_cast<const __nv_bfloat16 *>(gamma), static_cast<const __nv_bfloat16 *>(beta),
-        static_cast<__nv_bfloat16 *>(Y), rows, eps, out_row);
+    if (launch_pdl(vitk::layernorm_kernel, dim3(static_cast<unsigned>(blocks)), dim3(vitk::kLnWarps * 32), 0, s, 1, X,
+                   static_cast<const __nv_bfloat16 *>(gamma), static_cast<const __nv_bfloat16 *>(beta),
+                   static_cast<__nv_bfloat16 *>(Y), rows, eps, out_row) != cudaSuccess)
+        return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 
@@ -313,8 +318,9 @@ int positions_launch(const int32_t *grid_thw, int n_images, int64_t P, int patch
         row += static_cast<int64_t>(tab->t[i]) * tab->h[i] * tab->w[i];
     }
     if (P <= 0) return VIT_OK;
-    vitk::positions_kernel<<<static_cast<unsigned>((P + 255) / 256), 256, 0, s>>>(*tab, P, patch_order, pos,
-                                                                                 merge_row);
+    if (launch_pdl(vitk::positions_kernel, dim3(static_cast<unsigned>((P + 255) / 256)), dim3(256), 0, s, 1, *tab, P,
+                   patch_order, pos, merge_row) != cudaSuccess)
+        return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 
@@ -333,8 +339,9 @@ int positions_launch_stack(const int32_t *grid_thw, int n_images, int64_t P, int
         row += static_cast<int64_t>(tab.t[i]) * tab.h[i] * tab.w[i];
     }
     if (P <= 0) return VIT_OK;
-    vitk::positions_kernel<<<static_cast<unsigned>((P + 255) / 256), 256, 0, s>>>(tab, P, patch_order, pos,
-                                                                                 merge_row);
+    if (launch_pdl(vitk::positions_kernel, dim3(static_cast<unsigned>((P + 255) / 256)), dim3(256), 0, s, 1, tab, P,
+                   patch_order, pos, merge_row) != cudaSuccess)
+        return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 

@@ -388,6 +388,16 @@ __device__ __forceinline__ void exp2_fma2(float &x0, float &x1) {
     x1 = __int_as_float(max(static_cast<int>(__float_as_uint(t1) << 23) + __float_as_int(p1), 0));
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialisation (vith::launch_pdl) may start while the
+// previous kernel of its stream is still running: it sets up shared memory, barriers and tensor
+// memory meanwhile, and must not read or write global memory before pdl_wait(), which returns
+// once that kernel has completed and its writes are visible (a no-op in a kernel launched
+// without the attribute). pdl_trigger() allows the next kernel of the stream to start early; it
+// starts once every CTA of this grid has triggered or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

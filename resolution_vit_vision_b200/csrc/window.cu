@@ -101,6 +101,8 @@ __device__ __forceinline__ int last_le(const int *a, int n, int v) {   // last i
 __global__ void window_positions_kernel(const __grid_constant__ WinTable T, int64_t P, int patch_order,
                                         int32_t *__restrict__ pos, int32_t *__restrict__ merge_row,
                                         int32_t *__restrict__ src_row, int2 *__restrict__ win_tab) {
+    pdl_wait();                                   // the previous encode may still read these tables
+    pdl_trigger();
     const int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (r >= P) return;
     const int i = last_le(T.row_start, T.n_images, static_cast<int>(r));
@@ -124,6 +126,8 @@ __global__ void window_positions_kernel(const __grid_constant__ WinTable T, int6
 // dst[r, :] = src[src_row[r], :] for rows of `row_bytes` (a multiple of 16); one warp per row.
 __global__ void gather_rows_kernel(const uint4 *__restrict__ src, const int32_t *__restrict__ src_row,
                                    uint4 *__restrict__ dst, int64_t rows, int row_vecs) {
+    pdl_wait();                                   // src is the previous kernel's output
+    pdl_trigger();
     const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (r >= rows) return;
@@ -207,6 +211,10 @@ __global__ void __launch_bounds__(kWThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
+    // the previous kernel of the stream (the QKV product) has completed from here on; tensor
+    // memory is taken only after it
+    pdl_wait();
+    pdl_trigger();
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
@@ -447,8 +455,9 @@ int window_positions_launch(const int32_t *grid_thw, int n_images, int64_t P, in
     auto T = std::make_unique<vitk::WinTable>();
     fill_table(*T, grid_thw, n_images, window);
     if (P <= 0) return VIT_OK;
-    vitk::window_positions_kernel<<<static_cast<unsigned>((P + 255) / 256), 256, 0, s>>>(
-        *T, P, patch_order, pos, merge_row, src_row, reinterpret_cast<int2 *>(win_tab));
+    if (launch_pdl(vitk::window_positions_kernel, dim3(static_cast<unsigned>((P + 255) / 256)), dim3(256), 0, s, 1,
+                   *T, P, patch_order, pos, merge_row, src_row, reinterpret_cast<int2 *>(win_tab)) != cudaSuccess)
+        return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 
@@ -458,8 +467,10 @@ int gather_rows_launch(const void *src, const int32_t *src_row, void *dst, int64
         return VIT_ERR_ALIGN;
     if (rows <= 0) return VIT_OK;
     const int64_t threads = rows * 32;
-    vitk::gather_rows_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
-        static_cast<const uint4 *>(src), src_row, static_cast<uint4 *>(dst), rows, row_bytes / 16);
+    if (launch_pdl(vitk::gather_rows_kernel, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, s, 1,
+                   static_cast<const uint4 *>(src), src_row, static_cast<uint4 *>(dst), rows, row_bytes / 16) !=
+        cudaSuccess)
+        return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 
@@ -488,9 +499,10 @@ int win_attn_launch(const WinMaps &m, const int32_t *win_tab, int n_windows, int
     const int n_items = ((n_windows + 1) / 2) * VIT_HEADS;
     if (n_items == 0) return VIT_OK;
     const int grid = std::min(n_items, device_sm_count());
-    vitk::win_attn_kernel<<<grid, vitk::kWThreads, vitk::kWSmem, s>>>(
-        m.m32, m.m128, reinterpret_cast<const int2 *>(win_tab), n_windows, n_items, static_cast<int>(P),
-        static_cast<__nv_bfloat16 *>(out), status);
+    if (launch_pdl(vitk::win_attn_kernel, dim3(grid), dim3(vitk::kWThreads), vitk::kWSmem, s, 1, m.m32, m.m128,
+                   reinterpret_cast<const int2 *>(win_tab), n_windows, n_items, static_cast<int>(P),
+                   static_cast<__nv_bfloat16 *>(out), status) != cudaSuccess)
+        return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
 }
 
