@@ -22,6 +22,11 @@
  *     (the kernels read them with TMA); misaligned pointers return VIT_ERR_ALIGN.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
  *     default stream) except vit_device_status, which synchronises that stream.
+ *   - The encoder's kernels are launched with programmatic stream serialisation: each may start
+ *     while the stream's previous kernel drains, and waits for that kernel to complete before it
+ *     reads or writes any memory, so stream order holds for every caller. A kernel of the caller
+ *     launched next on the stream with the same attribute may likewise start early: it must wait
+ *     (griddepcontrol.wait / cudaGridDependencySynchronize) before reading the library's output.
  *   - Argument errors are returned synchronously, before anything is launched. Errors that
  *     depend on device data (a malformed M-RoPE prompt, a kernel wait that timed out) are
  *     written to a device status word and never trap.
