@@ -232,6 +232,31 @@ def test_graph_replay_matches_direct_launches():
     assert enc.device_status() == 0
 
 
+def test_back_to_back_encodes_on_one_stream():
+    # Different batches encoded one after another on one stream with nothing synchronising them:
+    # every kernel may start while its predecessor drains (programmatic dependent launch), so a
+    # kernel touching memory before its wait would let one encode read or overwrite another's
+    # positions, activations or output. Each result must equal the same batch encoded alone.
+    wts = syn.make_weights(2, 1536, 16)
+    enc = nv.VisionEncoder(nv.weights_to_device(wts), 1536)
+    batches = [[(1, 12, 16), (2, 4, 6)], [(1, 8, 8)], [(1, 20, 10), (1, 6, 6), (3, 4, 4)]]
+    ins = [bf16_bits_to_torch(syn.make_patches(g, 16 + i)) for i, g in enumerate(batches)]
+    refs = []
+    for p, g in zip(ins, batches):               # one at a time (this also grows the workspace)
+        refs.append(to_np(enc.encode(p, g)))
+    outs = [torch.full((r.shape[0], 1536), float("nan"), dtype=torch.bfloat16, device=DEV) for r in refs]
+    for graphs in (False, True):
+        enc.graph_enable(graphs)
+        for _ in range(3):
+            for p, g, o in zip(ins, batches, outs):
+                enc.encode(p, g, out=o)
+        torch.cuda.synchronize()
+        for o, r in zip(outs, refs):
+            np.testing.assert_array_equal(to_np(o), r)
+    enc.graph_enable(False)
+    assert enc.device_status() == 0
+
+
 @pytest.mark.slow
 def test_hires_1792_single_segment():
     # 16384 patches in one attention segment: the full depth-32 encode against the stored oracle
