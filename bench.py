@@ -259,7 +259,11 @@ def run_reference(args):
     full_blocks = tuple(int(x) for x in args.full_blocks.split(",") if x) if args.window else ()
     P, M4, _, _, _ = work_model(wl.grids, wl.depth, wl.out_dim, args.window, full_blocks)
     # each step: one bounded sample (the smallest image of the batch through the full-depth
-    # oracle); the run stops early once about three minutes of CPU time are spent
+    # oracle); one untimed sample first when warm-up steps are asked for (thread pools, first
+    # allocations); the run stops early once about three minutes of CPU time are spent
+    warm = min(args.warmup, 1)
+    for _ in range(warm):
+        cpu_baseline(wl, budget_s=20.0, window=args.window, full_blocks=full_blocks, fp8=args.fp8)
     vals = []
     t0 = time.perf_counter()
     for _ in range(max(1, args.steps)):
@@ -271,7 +275,7 @@ def run_reference(args):
     # a step here is the bounded sample, not the whole batch: ms_per_step is the sample's own
     # time; the whole batch at the sample's rate is reported separately as an extrapolation
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "patches/s", "n_gpus": args.gpus,
-            "steps": len(vals), "warmup": 0, "ms_per_step": sample_ms,
+            "steps": len(vals), "warmup": warm, "ms_per_step": sample_ms,
             "step_is": f"one bounded sample: {vals[0]['sample_patches']} patches of the batch through the "
                        f"full-depth oracle",
             "batch_ms_extrapolated": 1000.0 * P / v, "higher_is_better": True,
