@@ -15,10 +15,13 @@
 //   warp 1      (even CTA, one thread) MMA issuer: tcgen05.mma 256xBNx16 into the pair's TMEM
 //               accumulators, commits multicast to both CTAs; two accumulators so the epilogue of
 //               tile i overlaps the mainloop of tile i+1
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (one row per thread), bias,
-//               GELU / 2-D rope, then the tile leaves through a double-buffered swizzled shared
-//               staging chunk and a TMA store -- or a TMA reduce-add into the fp32 residual
-//               stream, so the residual update never reads the residual into the SM.
+//   warps 2..9  epilogue, two warpgroups that take every other column chunk (or head) of a
+//               tile: tcgen05.ld of the accumulator rows (one row per thread), bias, GELU / 2-D
+//               rope, then the chunk leaves through the group's swizzled shared staging buffer
+//               and a TMA store -- or a TMA reduce-add into the fp32 residual stream, so the
+//               residual update never reads the residual into the SM. Two groups halve the
+//               epilogue's time per tile, which the K = 1280 products (and all E4M3 products,
+//               whose mainloop runs at twice the rate) would otherwise wait on.
 // The same kernel runs the fp8 tower's products (F8 = true): A and B are E4M3 codes with a
 // power-of-two scale per row of A and per row of B ("Qwen2-VL-2B-Instruct -- LiteRT-LM", file
 // table: an 8-bit vision tower); a 128-byte k-block then holds 128 elements instead of 64, the
@@ -33,8 +36,9 @@ namespace vitk {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;           // 64 bf16 = 128 bytes: one 128B swizzle atom per row
-constexpr int kGemmThreads = 192;
-constexpr int kEpiBarrier = 1;    // named barrier of the 128 epilogue threads
+constexpr int kEpiGroups = 2;     // epilogue warpgroups, each takes every other column chunk of a tile
+constexpr int kGemmThreads = 64 + 128 * kEpiGroups;
+constexpr int kEpiBarrier = 1;    // named barriers kEpiBarrier + g of the 128 threads of group g
 
 template <int BN>
 struct GemmShape {
@@ -46,7 +50,7 @@ struct GemmShape {
     // output staging chunk: 128 rows x 128 bytes (32 fp32 or 64 bf16 columns), or for QKV one
     // 80-wide head as five 128 x 32-byte boxes
     static constexpr int STG_BYTES = BN == 240 ? 5 * 4096 : 16384;
-    static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + 2 * STG_BYTES + 256;
+    static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + kEpiGroups * STG_BYTES + 256;
     static_assert(B_BYTES % 1024 == 0, "B stage must keep 1024-byte alignment");
     static_assert(SMEM <= 232448, "shared memory per block");
 };
@@ -169,8 +173,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + S::STAGES * S::A_BYTES;
-    uint8_t *sStg = sB + S::STAGES * S::B_BYTES;            // [2][STG_BYTES], 1024-aligned
-    uint64_t *full = reinterpret_cast<uint64_t *>(sStg + 2 * S::STG_BYTES);
+    uint8_t *sStg = sB + S::STAGES * S::B_BYTES;            // [kEpiGroups][STG_BYTES], 1024-aligned
+    uint64_t *full = reinterpret_cast<uint64_t *>(sStg + kEpiGroups * S::STG_BYTES);
     uint64_t *empty = full + S::STAGES;
     uint64_t *tfull = empty + S::STAGES;
     uint64_t *tempty = tfull + 2;
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull + a, 1);
-            mbar_init(tempty + a, 8);                     // (CTA 0) the 4 + 4 epilogue warps of the pair
+            mbar_init(tempty + a, 8 * kEpiGroups);        // (CTA 0) every epilogue warp of the pair
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -265,19 +269,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
     } else {
+        const int grp = (warp - 2) >> 2;                        // epilogue group
         const int quarter = warp & 3;   // TMEM lanes [32*quarter, 32*quarter+32) belong to this warp
         const int r = quarter * 32 + lane;                      // row inside the tile
-        const bool leader = threadIdx.x == 64;                  // issues the TMA stores
+        const bool leader = threadIdx.x == 64 + 128 * grp;      // issues the group's TMA stores
         int sc = 0;                                             // staging chunks used so far
-        // Before filling staging buffer sc % 2, the store that last read it must be done.
+        // Each group has one staging buffer: before refilling it, the group's previous store must
+        // have read it.
         auto stage_acquire = [&]() {
-            if (leader && sc >= 2) bulk_wait_read<1>();
-            named_bar_sync(kEpiBarrier, 128);
-            return sStg + (sc & 1) * S::STG_BYTES;
+            if (leader && sc >= 1) bulk_wait_read<0>();
+            named_bar_sync(kEpiBarrier + grp, 128);
+            return sStg + grp * S::STG_BYTES;
         };
         auto stage_publish = [&]() {
             fence_proxy_async_smem();
-            named_bar_sync(kEpiBarrier, 128);
+            named_bar_sync(kEpiBarrier + grp, 128);
         };
         const uint32_t tempty0 = cluster_addr(tempty, 0);   // CTA 0's accumulator-free barriers
         // this warp's share of the accumulator is read: one arrival per warp on CTA 0's barrier
@@ -296,14 +302,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t t0 = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * S::ACC_STRIDE;
             if (EPI == VIT_EPI_QKV_ROPE) {
 #pragma unroll 1
-                for (int hh = 0; hh < BN / 80; ++hh) {
+                for (int hh = grp; hh < BN / 80; hh += kEpiGroups) {
                     uint32_t u[80];
 #pragma unroll
                     for (int c = 0; c < 5; ++c) tmem_ld16(t0 + hh * 80 + c * 16, u + c * 16);
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 5; ++c) reg_fence16(u + c * 16);
-                    if (hh == BN / 80 - 1) release_acc(acc);   // accumulator fully read: hand it back
+                    if (hh + kEpiGroups >= BN / 80) release_acc(acc);   // this warp's reads are done
                     float v[80];
 #pragma unroll
                     for (int j = 0; j < 80; ++j) v[j] = __uint_as_float(u[j]);
@@ -336,12 +342,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             } else if (EPI == VIT_EPI_STORE_F32 || EPI == VIT_EPI_ADD_F32) {
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {     // 32 fp32 columns = one 128-byte row per chunk
+                for (int c = grp; c < BN / 32; c += kEpiGroups) {   // 32 fp32 columns = a 128-byte row
                     uint32_t u[32];
                     tmem_ld32(t0 + c * 32, u);
                     tmem_wait_ld();
                     reg_fence32(u);
-                    if (c == BN / 32 - 1) release_acc(acc);
+                    if (c + kEpiGroups >= BN / 32) release_acc(acc);
                     const int col0 = n0 + c * 32;
                     if (col0 < p.N) {                   // uniform across the CTA
                         float v[32];
@@ -364,14 +370,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < BN / 64; ++c) {     // 64 bf16 columns = one 128-byte row per chunk
+                for (int c = grp; c < BN / 64; c += kEpiGroups) {   // 64 bf16 columns = a 128-byte row
                     uint32_t u[64];
                     tmem_ld32(t0 + c * 64, *reinterpret_cast<uint32_t(*)[32]>(u));
                     tmem_ld32(t0 + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
                     tmem_wait_ld();
                     reg_fence32(u);
                     reg_fence32(u + 32);
-                    if (c == BN / 64 - 1) release_acc(acc);
+                    if (c + kEpiGroups >= BN / 64) release_acc(acc);
                     const int col0 = n0 + c * 64;
                     if (col0 < p.N) {
                         float v[64];
