@@ -37,6 +37,7 @@ GEMM_CASES = [
     (200, 304, 72),
     (4800, 1280, 1280),      # enough 256 x 256 tiles to fill the SM pairs: the wide tiles
     (2100, 5120, 1280),
+    (2100, 1328, 1280),      # wide tiles with an N tail: the two epilogue groups get unequal chunks
 ]
 
 
