@@ -15,13 +15,13 @@
 //   warp 1      (even CTA, one thread) MMA issuer: tcgen05.mma 256xBNx16 into the pair's TMEM
 //               accumulators, commits multicast to both CTAs; two accumulators so the epilogue of
 //               tile i overlaps the mainloop of tile i+1
-//   warps 2..9  epilogue, two warpgroups that take every other column chunk (or head) of a
-//               tile: tcgen05.ld of the accumulator rows (one row per thread), bias, GELU / 2-D
-//               rope, then the chunk leaves through the group's swizzled shared staging buffer
-//               and a TMA store -- or a TMA reduce-add into the fp32 residual stream, so the
-//               residual update never reads the residual into the SM. Two groups halve the
-//               epilogue's time per tile, which the K = 1280 products (and all E4M3 products,
-//               whose mainloop runs at twice the rate) would otherwise wait on.
+//   warps 2..5  epilogue (and 6..9: a second warpgroup for the products whose epilogue would
+//               otherwise hold the mainloop back -- E4M3, rope, small-batch tiles -- each group
+//               taking every other column chunk or head of a tile): tcgen05.ld of the
+//               accumulator rows (one row per thread), bias, GELU / 2-D rope, then the chunk
+//               leaves through a swizzled shared staging buffer and a TMA store -- or a TMA
+//               reduce-add into the fp32 residual stream, so the residual update never reads the
+//               residual into the SM.
 // The same kernel runs the fp8 tower's products (F8 = true): A and B are E4M3 codes with a
 // power-of-two scale per row of A and per row of B ("Qwen2-VL-2B-Instruct -- LiteRT-LM", file
 // table: an 8-bit vision tower); a 128-byte k-block then holds 128 elements instead of 64, the
@@ -36,9 +36,18 @@ namespace vitk {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;           // 64 bf16 = 128 bytes: one 128B swizzle atom per row
-constexpr int kEpiGroups = 2;     // epilogue warpgroups, each takes every other column chunk of a tile
-constexpr int kGemmThreads = 64 + 128 * kEpiGroups;
 constexpr int kEpiBarrier = 1;    // named barriers kEpiBarrier + g of the 128 threads of group g
+
+// Epilogue warpgroups of a product: two, each taking every other column chunk (or head) of a tile,
+// where the epilogue would otherwise hold the mainloop back -- the E4M3 products (twice the
+// product rate), the rope epilogue, the 256 x 128 tiles of small batches -- else one. The two
+// staging buffers are double-buffered by one group or split between two.
+template <int BN, int EPI, bool F8>
+struct GemmCfg {
+    static constexpr int GROUPS = (F8 || EPI == VIT_EPI_QKV_ROPE || BN == 128) ? 2 : 1;
+    static constexpr int THREADS = 64 + 128 * GROUPS;
+    static constexpr int NBUF = 2 / GROUPS;   // staging buffers per group
+};
 
 template <int BN>
 struct GemmShape {
@@ -50,7 +59,7 @@ struct GemmShape {
     // output staging chunk: 128 rows x 128 bytes (32 fp32 or 64 bf16 columns), or for QKV one
     // 80-wide head as five 128 x 32-byte boxes
     static constexpr int STG_BYTES = BN == 240 ? 5 * 4096 : 16384;
-    static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + kEpiGroups * STG_BYTES + 256;
+    static constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + 2 * STG_BYTES + 256;
     static_assert(B_BYTES % 1024 == 0, "B stage must keep 1024-byte alignment");
     static_assert(SMEM <= 232448, "shared memory per block");
 };
@@ -165,16 +174,17 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
 }
 
 template <int BN, int EPI, bool F8>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(GemmCfg<BN, EPI, F8>::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                    const __grid_constant__ CUtensorMap tmc, GemmParams p) {
     using S = GemmShape<BN>;
+    using C = GemmCfg<BN, EPI, F8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + S::STAGES * S::A_BYTES;
-    uint8_t *sStg = sB + S::STAGES * S::B_BYTES;            // [kEpiGroups][STG_BYTES], 1024-aligned
-    uint64_t *full = reinterpret_cast<uint64_t *>(sStg + kEpiGroups * S::STG_BYTES);
+    uint8_t *sStg = sB + S::STAGES * S::B_BYTES;            // [2][STG_BYTES], 1024-aligned
+    uint64_t *full = reinterpret_cast<uint64_t *>(sStg + 2 * S::STG_BYTES);
     uint64_t *empty = full + S::STAGES;
     uint64_t *tfull = empty + S::STAGES;
     uint64_t *tempty = tfull + 2;
@@ -191,7 +201,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull + a, 1);
-            mbar_init(tempty + a, 8 * kEpiGroups);        // (CTA 0) every epilogue warp of the pair
+            mbar_init(tempty + a, 8 * C::GROUPS);         // (CTA 0) every epilogue warp of the pair
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -274,12 +284,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int r = quarter * 32 + lane;                      // row inside the tile
         const bool leader = threadIdx.x == 64 + 128 * grp;      // issues the group's TMA stores
         int sc = 0;                                             // staging chunks used so far
-        // Each group has one staging buffer: before refilling it, the group's previous store must
-        // have read it.
+        // Before refilling one of the group's staging buffers, the store that last read it must be
+        // done.
         auto stage_acquire = [&]() {
-            if (leader && sc >= 1) bulk_wait_read<0>();
+            if (leader && sc >= C::NBUF) bulk_wait_read<C::NBUF - 1>();
             named_bar_sync(kEpiBarrier + grp, 128);
-            return sStg + grp * S::STG_BYTES;
+            return sStg + (grp * C::NBUF + sc % C::NBUF) * S::STG_BYTES;
         };
         auto stage_publish = [&]() {
             fence_proxy_async_smem();
@@ -302,14 +312,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t t0 = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * S::ACC_STRIDE;
             if (EPI == VIT_EPI_QKV_ROPE) {
 #pragma unroll 1
-                for (int hh = grp; hh < BN / 80; hh += kEpiGroups) {
+                for (int hh = grp; hh < BN / 80; hh += C::GROUPS) {
                     uint32_t u[80];
 #pragma unroll
                     for (int c = 0; c < 5; ++c) tmem_ld16(t0 + hh * 80 + c * 16, u + c * 16);
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 5; ++c) reg_fence16(u + c * 16);
-                    if (hh + kEpiGroups >= BN / 80) release_acc(acc);   // this warp's reads are done
+                    if (hh + C::GROUPS >= BN / 80) release_acc(acc);   // this warp's reads are done
                     float v[80];
 #pragma unroll
                     for (int j = 0; j < 80; ++j) v[j] = __uint_as_float(u[j]);
@@ -342,12 +352,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             } else if (EPI == VIT_EPI_STORE_F32 || EPI == VIT_EPI_ADD_F32) {
 #pragma unroll 1
-                for (int c = grp; c < BN / 32; c += kEpiGroups) {   // 32 fp32 columns = a 128-byte row
+                for (int c = grp; c < BN / 32; c += C::GROUPS) {   // 32 fp32 columns = a 128-byte row
                     uint32_t u[32];
                     tmem_ld32(t0 + c * 32, u);
                     tmem_wait_ld();
                     reg_fence32(u);
-                    if (c + kEpiGroups >= BN / 32) release_acc(acc);
+                    if (c + C::GROUPS >= BN / 32) release_acc(acc);
                     const int col0 = n0 + c * 32;
                     if (col0 < p.N) {                   // uniform across the CTA
                         float v[32];
@@ -370,14 +380,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             } else {
 #pragma unroll 1
-                for (int c = grp; c < BN / 64; c += kEpiGroups) {   // 64 bf16 columns = a 128-byte row
+                for (int c = grp; c < BN / 64; c += C::GROUPS) {   // 64 bf16 columns = a 128-byte row
                     uint32_t u[64];
                     tmem_ld32(t0 + c * 64, *reinterpret_cast<uint32_t(*)[32]>(u));
                     tmem_ld32(t0 + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
                     tmem_wait_ld();
                     reg_fence32(u);
                     reg_fence32(u + 32);
-                    if (c + kEpiGroups >= BN / 64) release_acc(acc);
+                    if (c + C::GROUPS >= BN / 64) release_acc(acc);
                     const int col0 = n0 + c * 64;
                     if (col0 < p.N) {
                         float v[64];
@@ -466,6 +476,7 @@ template <int BN, int EPI, bool F8>
 static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc, const vitk::GemmParams &p,
                       cudaStream_t s) {
     using S = vitk::GemmShape<BN>;
+    using C = vitk::GemmCfg<BN, EPI, F8>;
     static bool configured[64] = {};   // the attribute is set once per device
     int dev = 0;
     cudaGetDevice(&dev);
@@ -483,7 +494,7 @@ static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtens
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
-        cfg.blockDim = dim3(vitk::kGemmThreads);
+        cfg.blockDim = dim3(C::THREADS);
         cfg.dynamicSmemBytes = S::SMEM;
         cfg.stream = s;
         cfg.attrs = attr;
@@ -499,7 +510,7 @@ static int launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtens
     const int total = p.m_tiles * p.n_tiles;
     const int pairs = dev < 64 ? max_clusters[dev] : device_sm_count() / 2;
     const dim3 grid(2 * (total < pairs ? total : pairs));
-    if (launch_pdl(vitk::gemm_tc_kernel<BN, EPI, F8>, grid, dim3(vitk::kGemmThreads), S::SMEM, s, 2, ta, tb, tc, p) !=
+    if (launch_pdl(vitk::gemm_tc_kernel<BN, EPI, F8>, grid, dim3(C::THREADS), S::SMEM, s, 2, ta, tb, tc, p) !=
         cudaSuccess)
         return VIT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VIT_OK : VIT_ERR_CUDA;
